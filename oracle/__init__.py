@@ -1,0 +1,158 @@
+"""CPU fp64 oracle for block-sparse GQA attention with a mean-pooled block cache.
+
+TEST INFRASTRUCTURE ONLY: the test suite, the package's smoke check and the
+benchmark's CPU-baseline leg are the only callers. The product path (the CUDA
+library and its Python binding) never imports this package.
+
+The arithmetic lives in ``msa_oracle.cpp`` (plain C++17 + OpenMP, fp64). This
+module converts arrays and calls it. Every function takes the *logical*
+(unpaged) tensors of one sequence:
+
+  K, V : [L, Hkv, d]     keys / values at positions 0 .. L-1
+  Q    : [R, Hq, d]      query rows, row r at position pos[r]
+
+as fp32 arrays or bf16 bit patterns (torch.bfloat16 tensors or uint16 numpy
+arrays); elements are widened to double on use.
+
+Citations (page title, section):
+  * centroids  - "Art of Focus: Ling 2.0 ...", "Summarizing the Breakthrough":
+                 blocks are aggregated into representations kept in the cache
+                 (read here as the mean of the keys present).
+  * scores, select - "MiniMax Sparse Attention", method paragraph: the index
+                 branch scores KV blocks and takes a top-k subset per GQA group;
+                 results paragraph: the top-k is exp-free.
+  * attend     - "MiniMax Sparse Attention", method paragraph (exact blockwise
+                 sparse attention over the chosen blocks) and "Sparse Attention
+                 + Linear Backbones", section 5.5 (softmax(q k^T / sqrt(d)) v).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Dict
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "msa_oracle.cpp")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_I32 = ctypes.c_int
+
+
+def build(force: bool = False) -> str:
+    """Compile liboracle.so next to its source (g++, -O2, OpenMP)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["g++", "-O2", "-std=c++17", "-fopenmp", "-fPIC", "-shared",
+                               "-o", tmp, _SRC])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        lib.orc_centroids.restype = _I64
+        lib.orc_centroids.argtypes = [_P, _I32, _I64, _I32, _I32, _I32, _P]
+        lib.orc_scores.restype = None
+        lib.orc_scores.argtypes = [_P, _I32, _I64, _P, _I32, _I32, _I32, _I32, _P, _I64, _P]
+        lib.orc_select.restype = None
+        lib.orc_select.argtypes = [_P, _I64, _P, _I32, _I64, _I32, _I32, _P, _P]
+        lib.orc_attend.restype = None
+        lib.orc_attend.argtypes = [_P, _P, _P, _I32, _I64, _P, _I64, _I32, _I32, _I32, _I32, _P,
+                                   _I32, ctypes.c_double, _P, _P]
+        lib.orc_num_threads.restype = _I32
+        _lib = lib
+    return _lib
+
+
+def num_threads() -> int:
+    return int(_load().orc_num_threads())
+
+
+def _elems(x):
+    """(contiguous numpy array, dtype code) for fp32 or bf16-bit input."""
+    try:
+        import torch
+        if isinstance(x, torch.Tensor):
+            x = x.detach().cpu().contiguous()
+            if x.dtype == torch.bfloat16:
+                return np.ascontiguousarray(x.view(torch.int16).numpy().view(np.uint16)), 1
+            return np.ascontiguousarray(x.to(torch.float32).numpy()), 0
+    except ImportError:  # pragma: no cover
+        pass
+    x = np.asarray(x)
+    if x.dtype == np.uint16:
+        return np.ascontiguousarray(x), 1
+    return np.ascontiguousarray(x, dtype=np.float32), 0
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def centroids(K, block: int) -> np.ndarray:
+    """[ceil(L/B), Hkv, d] fp64 mean of the keys present in each block."""
+    k, dt = _elems(K)
+    L, hkv, d = k.shape
+    nblk = -(-L // block)
+    C = np.empty((nblk, hkv, d), dtype=np.float64)
+    _load().orc_centroids(_ptr(k), dt, L, hkv, d, block, _ptr(C))
+    return C
+
+
+def scores(Q, pos, C: np.ndarray, block: int) -> np.ndarray:
+    """[R, Hkv, nblk] fp64 block scores; NaN outside the candidate set."""
+    q, dt = _elems(Q)
+    R, hq, d = q.shape
+    nblk, hkv, _ = C.shape
+    pos = np.ascontiguousarray(pos, dtype=np.int64)
+    C = np.ascontiguousarray(C, dtype=np.float64)
+    S = np.empty((R, hkv, nblk), dtype=np.float64)
+    _load().orc_scores(_ptr(q), dt, R, _ptr(pos), hq, hkv, d, block, _ptr(C), nblk, _ptr(S))
+    return S
+
+
+def select(S: np.ndarray, pos, block: int, top_k: int):
+    """(idx [R, Hkv, k] int32 ascending, -1 padded; gap [R, Hkv] fp64)."""
+    S = np.ascontiguousarray(S, dtype=np.float64)
+    R, hkv, nblk = S.shape
+    pos = np.ascontiguousarray(pos, dtype=np.int64)
+    idx = np.empty((R, hkv, top_k), dtype=np.int32)
+    gap = np.empty((R, hkv), dtype=np.float64)
+    _load().orc_select(_ptr(S), R, _ptr(pos), hkv, nblk, block, top_k, _ptr(idx), _ptr(gap))
+    return idx, gap
+
+
+def attend(Q, K, V, pos, idx, block: int, scale: float):
+    """(O [R, Hq, d] fp64, lse [R, Hq] fp64) of exact attention over idx's blocks."""
+    q, dq = _elems(Q)
+    k, dk = _elems(K)
+    v, dv = _elems(V)
+    if not (dq == dk == dv):
+        raise TypeError("Q, K, V must share one element type")
+    R, hq, d = q.shape
+    L, hkv, _ = k.shape
+    pos = np.ascontiguousarray(pos, dtype=np.int64)
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    top_k = idx.shape[-1]
+    O = np.empty((R, hq, d), dtype=np.float64)
+    lse = np.empty((R, hq), dtype=np.float64)
+    _load().orc_attend(_ptr(q), _ptr(k), _ptr(v), dq, R, _ptr(pos), L, hq, hkv, d, block,
+                       _ptr(idx), top_k, float(scale), _ptr(O), _ptr(lse))
+    return O, lse
+
+
+def forward(Q, K, V, pos, block: int, top_k: int, scale: float) -> Dict[str, np.ndarray]:
+    """Whole path for one sequence: centroids -> scores -> top-k -> attention."""
+    C = centroids(K, block)
+    S = scores(Q, pos, C, block)
+    idx, gap = select(S, pos, block, top_k)
+    O, lse = attend(Q, K, V, pos, idx, block, scale)
+    return {"centroids": C, "scores": S, "idx": idx, "gap": gap, "out": O, "lse": lse}

@@ -1,0 +1,266 @@
+"""Pins for the CPU oracle: each check ties it to something other than itself.
+
+* library routines: torch's scaled_dot_product_attention and logsumexp (CPU,
+  float64) for the cases where the method reduces to dense or block-local
+  causal attention;
+* closed forms: centroids of a ramp of keys, scores of one-hot queries, the
+  selection and gap of monotone score ramps;
+* brute force: enumeration of every candidate subset on tiny inputs;
+* invariants: softmax weights are non-negative, sum to one and vanish off the
+  attended set; one-key rows return that key's value exactly.
+
+The method: "MiniMax Sparse Attention" (staik.se), method paragraph (per-GQA-
+group top-k over KV blocks, then exact attention over them); "Art of Focus:
+Ling 2.0 ...", "Summarizing the Breakthrough" (block representations in a
+cache, GQA-shared selection); "Sparse Attention + Linear Backbones", section
+5.5 (softmax(q k^T / sqrt(d)) v over the selected set).
+"""
+import itertools
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+
+
+def _rand(shape, seed, dtype=torch.float32):
+    g = torch.Generator().manual_seed(seed)
+    return torch.randn(*shape, generator=g, dtype=torch.float64).to(dtype)
+
+
+def _sdpa_ref(Q, K, V, mask, scale):
+    """torch SDPA in float64 with K/V heads repeated for GQA. mask: [R, L] bool."""
+    G = Q.shape[1] // K.shape[1]
+    q = Q.to(torch.float64).permute(1, 0, 2)                       # [Hq, R, d]
+    k = K.to(torch.float64).repeat_interleave(G, dim=1).permute(1, 0, 2)
+    v = V.to(torch.float64).repeat_interleave(G, dim=1).permute(1, 0, 2)
+    o = torch.nn.functional.scaled_dot_product_attention(q, k, v, attn_mask=mask, scale=scale)
+    return o.permute(1, 0, 2).numpy()
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("L,B,d,hq,hkv", [(200, 16, 32, 6, 2), (97, 8, 16, 4, 4), (64, 64, 64, 4, 1)])
+def test_dense_pin(dtype, L, B, d, hq, hkv):
+    """k >= number of blocks: the method is dense causal attention."""
+    Q, K, V = _rand((L, hq, d), 1, dtype), _rand((L, hkv, d), 2, dtype), _rand((L, hkv, d), 3, dtype)
+    nblk = -(-L // B)
+    pos = np.arange(L)
+    scale = 1.0 / math.sqrt(d)
+    r = oracle.forward(Q, K, V, pos, B, nblk + 1, scale)
+    causal = torch.ones(L, L, dtype=torch.bool).tril()
+    ref = _sdpa_ref(Q, K, V, causal, scale)
+    assert np.max(np.abs(r["out"] - ref)) < 1e-12
+    # lse against the library logsumexp of the masked logits
+    G = hq // hkv
+    logits = torch.einsum("rhd,uhd->hru", Q.to(torch.float64),
+                          K.to(torch.float64).repeat_interleave(G, dim=1)) * scale
+    logits = logits.masked_fill(~causal, float("-inf"))
+    lse_ref = torch.logsumexp(logits, dim=-1).T.numpy()
+    assert np.max(np.abs(r["lse"] - lse_ref)) < 1e-10
+
+
+@pytest.mark.parametrize("L,B", [(130, 16), (64, 8)])
+def test_block_local_pin(L, B):
+    """k = 1: each query attends causally inside its own block only."""
+    d, hq, hkv = 24, 4, 2
+    Q, K, V = _rand((L, hq, d), 4), _rand((L, hkv, d), 5), _rand((L, hkv, d), 6)
+    pos = np.arange(L)
+    scale = 1.0 / math.sqrt(d)
+    r = oracle.forward(Q, K, V, pos, B, 1, scale)
+    t = torch.arange(L)
+    mask = (t[None, :] <= t[:, None]) & ((t[None, :] // B) == (t[:, None] // B))
+    ref = _sdpa_ref(Q, K, V, mask, scale)
+    assert np.max(np.abs(r["out"] - ref)) < 1e-12
+    # rows that open a block see exactly one key: output is that value, exactly
+    for t0 in range(0, L, B):
+        for h in range(hq):
+            assert np.array_equal(r["out"][t0, h], V[t0, h // (hq // hkv)].to(torch.float64).numpy())
+
+
+def test_softmax_weights():
+    """One-hot values expose the weights: >= 0, sum to 1, zero off the attended set."""
+    L, B, d, hq, hkv, k = 40, 5, 64, 2, 1, 3
+    Q, K = _rand((L, hq, d), 7) * 2.0, _rand((L, hkv, d), 8)
+    V = torch.zeros(L, hkv, d)
+    for u in range(L):
+        V[u, 0, u] = 1.0
+    pos = np.arange(L)
+    r = oracle.forward(Q, K, V, pos, B, k, 0.125)
+    W = r["out"][:, :, :L]
+    assert np.all(W >= 0)
+    assert np.max(np.abs(W.sum(-1) - 1.0)) < 1e-12
+    for t in range(L):
+        allowed = set()
+        for j in r["idx"][t, 0]:
+            if j >= 0:
+                allowed |= {u for u in range(j * B, (j + 1) * B) if u <= t}
+        off = [u for u in range(L) if u not in allowed]
+        assert np.all(W[t, :, off] == 0.0)
+
+
+def test_centroid_closed_form():
+    """Keys k[u] = u * e1 give c_j = (jB + (n_j - 1)/2) e1, n_j tokens present."""
+    L, B, d = 203, 16, 8
+    K = torch.zeros(L, 2, d)
+    K[:, :, 0] = torch.arange(L, dtype=torch.float32)[:, None]
+    C = oracle.centroids(K, B)
+    assert C.shape == (13, 2, d)
+    for j in range(13):
+        n = min(B, L - j * B)
+        assert C[j, 0, 0] == j * B + (n - 1) / 2.0
+        assert C[j, 1, 0] == j * B + (n - 1) / 2.0
+        assert np.all(C[j, :, 1:] == 0.0)
+
+
+def test_scores_one_hot_queries():
+    """One-hot queries pick centroid coordinates: s_j = sum_h c_j[i_h]; NaN if j >= b(t)."""
+    L, B, d, hq, hkv = 64, 8, 6, 4, 2
+    K = _rand((L, hkv, d), 9)
+    C = oracle.centroids(K, B)
+    Q = torch.zeros(3, hq, d)
+    hot = [[0, 5, 2, 2], [1, 1, 4, 3], [3, 0, 0, 5]]
+    for r in range(3):
+        for h in range(hq):
+            Q[r, h, hot[r][h]] = 1.0
+    pos = np.array([63, 40, 17])
+    S = oracle.scores(Q, pos, C, B)
+    for r in range(3):
+        bt = pos[r] // B
+        for g in range(hkv):
+            for j in range(C.shape[0]):
+                if j >= bt:
+                    assert np.isnan(S[r, g, j])
+                else:
+                    want = C[j, g, hot[r][2 * g]] + C[j, g, hot[r][2 * g + 1]]
+                    assert abs(S[r, g, j] - want) < 1e-15
+
+
+def _brute_force(scores_row, bt, k):
+    """Best (k-1)-subset of past blocks under (score desc, index asc) - by enumeration."""
+    take = min(k - 1, bt)
+    best = None
+    for comb in itertools.combinations(range(bt), take):
+        keylist = sorted(((scores_row[j], -j) for j in comb), reverse=True)
+        if best is None or keylist > best[0]:
+            best = (keylist, comb)
+    chosen = sorted(set(best[1]) | {bt})
+    rejected = [scores_row[j] for j in range(bt) if j not in best[1]]
+    gap = (min(scores_row[j] for j in best[1]) - max(rejected)) if (take > 0 and rejected) else math.inf
+    return chosen, gap
+
+
+@pytest.mark.parametrize("k", [1, 2, 3, 4])
+def test_selection_brute_force(k):
+    L, B, d, hq, hkv = 44, 4, 8, 4, 2
+    Q, K = _rand((L, hq, d), 10 + k), _rand((L, hkv, d), 20 + k)
+    pos = np.arange(L)
+    C = oracle.centroids(K, B)
+    S = oracle.scores(Q, pos, C, B)
+    idx, gap = oracle.select(S, pos, B, k)
+    for t in range(L):
+        for g in range(hkv):
+            chosen, bgap = _brute_force(S[t, g], t // B, k)
+            got = [int(j) for j in idx[t, g] if j >= 0]
+            assert got == chosen
+            assert list(idx[t, g][len(got):]) == [-1] * (k - len(got))
+            if math.isinf(bgap):
+                assert math.isinf(gap[t, g])
+            else:
+                assert abs(gap[t, g] - bgap) < 1e-14
+
+
+def test_exact_ties_go_to_lower_index():
+    """Duplicated blocks score bit-identically; the lower index wins the last slot."""
+    L, B, d, hq, hkv, k = 64, 8, 4, 2, 1, 3
+    K = torch.zeros(L, hkv, d)
+    K[:, 0, 0] = -1.0
+    for j in (2, 5):            # two identical high-scoring blocks
+        K[j * B:(j + 1) * B, 0, 0] = 3.0
+    K[1 * B:2 * B, 0, 0] = 5.0  # one clear winner
+    Q = torch.zeros(1, hq, d)
+    Q[0, :, 0] = 1.0
+    pos = np.array([L - 1])
+    C = oracle.centroids(K, B)
+    S = oracle.scores(Q, pos, C, B)
+    assert S[0, 0, 2] == S[0, 0, 5]
+    idx, gap = oracle.select(S, pos, B, k)
+    assert list(idx[0, 0]) == [1, 2, 7]
+    assert gap[0, 0] == 0.0
+
+
+def test_all_equal_scores_pick_lowest():
+    L, B, d, k = 80, 8, 4, 4
+    K = torch.zeros(L, 1, d)
+    Q = torch.ones(5, 2, d)
+    pos = np.array([79, 70, 31, 24, 8])
+    S = oracle.scores(Q, pos, oracle.centroids(K, B), B)
+    idx, _ = oracle.select(S, pos, B, k)
+    assert list(idx[0, 0]) == [0, 1, 2, 9]
+    assert list(idx[1, 0]) == [0, 1, 2, 8]
+    assert list(idx[2, 0]) == [0, 1, 2, 3]   # b = 3 = k-1: every past block kept
+    assert list(idx[3, 0]) == [0, 1, 2, 3]
+    assert list(idx[4, 0]) == [0, 1, -1, -1]
+
+
+@pytest.mark.parametrize("sign", [1.0, -1.0])
+def test_score_ramp_closed_form(sign):
+    """Block-constant keys sign*j*e1 and queries e1: scores sign*G*j. An increasing
+    ramp keeps the k-1 latest past blocks (never a future one), a decreasing ramp
+    the k-1 earliest; the gap is G either way."""
+    L, B, d, hq, hkv, k = 160, 8, 4, 6, 2, 5
+    G = hq // hkv
+    K = torch.zeros(L, hkv, d)
+    K[:, :, 0] = sign * (torch.arange(L) // B).to(torch.float32)[:, None]
+    Q = torch.zeros(L, hq, d)
+    Q[:, :, 0] = 1.0
+    pos = np.arange(L)
+    S = oracle.scores(Q, pos, oracle.centroids(K, B), B)
+    idx, gap = oracle.select(S, pos, B, k)
+    for t in range(L):
+        b = t // B
+        for g in range(hkv):
+            if b < k:
+                want = list(range(b + 1)) + [-1] * (k - b - 1)
+            elif sign > 0:
+                want = list(range(b - k + 1, b + 1))
+            else:
+                want = list(range(k - 1)) + [b]
+            assert list(idx[t, g]) == want
+            if b >= k:
+                assert gap[t, g] == G
+            else:
+                assert math.isinf(gap[t, g])
+
+
+def test_permuted_index_order_and_row_subsets():
+    """Attention does not depend on the order of the index list, and a row
+    computed alone equals the same row computed with all others."""
+    L, B, d, hq, hkv, k = 96, 8, 16, 4, 2, 4
+    Q, K, V = _rand((L, hq, d), 30), _rand((L, hkv, d), 31), _rand((L, hkv, d), 32)
+    pos = np.arange(L)
+    r = oracle.forward(Q, K, V, pos, B, k, 0.25)
+    perm_idx = r["idx"][:, :, ::-1].copy()
+    O2, lse2 = oracle.attend(Q, K, V, pos, perm_idx, B, 0.25)
+    assert np.max(np.abs(O2 - r["out"])) < 1e-13
+    one = oracle.forward(Q[L - 1:], K, V, pos[L - 1:], B, k, 0.25)
+    assert np.array_equal(one["idx"][0], r["idx"][L - 1])
+    assert np.max(np.abs(one["out"][0] - r["out"][L - 1])) < 1e-15
+
+
+def test_tiny_workload_finds_planted_blocks():
+    """Generator + oracle: the tiny workload plants two blocks along the last
+    query's mean head direction, so that query ranks them first."""
+    w = workloads.tiny_f32()
+    L = w.ctx[0]
+    K = workloads.keys(w, 0, 0, L)
+    V = workloads.values(w, 0, 0, L)
+    Q = workloads.queries_prefill(w, 0, 0, L)
+    planted = workloads.planted_blocks(w)[0][0]
+    assert len(planted) == 2 and all(j < 15 for j in planted)
+    r = oracle.forward(Q[L - 1:], K, V, np.array([L - 1]), w.block, w.top_k, w.softmax_scale)
+    S = r["scores"][0, 0, :L // w.block - 1]
+    assert sorted(np.argsort(-S)[:2].tolist()) == planted
+    assert set(planted) <= set(int(j) for j in r["idx"][0, 0])
