@@ -1,0 +1,578 @@
+"""Benchmark of the block-sparse GQA attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+                    [--workload prefill_bf16|paged_decode_bf16|decode_1m_bf16|varlen_decode_bf16]
+
+A step is one pass of the whole hot path over one batch of synthetic input:
+  prefill workloads : KV append with centroid pooling (msa_build_block_cache),
+                      top-k selection (msa_select_topk) and sparse attention
+                      (msa_sparse_attn_prefill) over all query rows;
+  decode workloads  : append of one token per sequence, decode selection and
+                      split-k decode attention.
+The default workload is the prefill one (batch 1, 32768 tokens, 32/4 heads,
+d 128, block 128, top-k 16); a paged-decode block (batch 32, 131072 cached
+tokens, 32/8 heads, block 64, top-k 32) is measured in the same run.
+
+Timing: W untimed warm-up steps, then K steps between a barrier and
+torch.cuda.synchronize() on both sides, CUDA events on the launching stream,
+max over ranks. Inputs of every step exceed the 126 MB L2 (prefill: 0.7 GB;
+paged decode: ~0.53 GB read per step); the 1M-context decode working set
+(~42 MB) does not, so that workload writes a 256 MB buffer between steps.
+Under torchrun each rank runs its own replica of the workload (independent
+sequences, no collective on the data path): weak scaling.
+
+--impl reference times the CPU fp64 oracle (the reference arm) on a bounded
+sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "sparse-attn decode tokens/s + HBM GB/s; prefill tokens/s + tensor-pipe util"
+
+
+# ---------------------------------------------------------------------------
+# helpers
+# ---------------------------------------------------------------------------
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def profile_traffic(kernel: str, src: str):
+    """ncu DRAM bytes per launch recorded in profiles/<kernel>*.md, if the kernel
+    source still hashes to the recorded value; else None."""
+    pdir = os.path.join(ROOT, "profiles")
+    sha = hashlib.sha256(open(os.path.join(ROOT, "block_sparse_gqa_mean_b200", "csrc", src),
+                              "rb").read()).hexdigest()[:16]
+    if not os.path.isdir(pdir):
+        return None
+    for f in sorted(os.listdir(pdir)):
+        if not (f.startswith(kernel) and f.endswith(".md")):
+            continue
+        vals = {}
+        for line in open(os.path.join(pdir, f)):
+            if ":" in line and line.strip().startswith(("source_sha256", "dram_bytes_per_full_launch")):
+                k, v = line.strip().split(":", 1)
+                vals[k.strip()] = v.strip().strip("`")
+        if vals.get("source_sha256") == sha and "dram_bytes_per_full_launch" in vals:
+            return float(vals["dram_bytes_per_full_launch"])
+    return None
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"msa_clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = [r.split(",") for r in open(self.path).read().strip().splitlines() if r.count(",") >= 8]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows]
+        smax = max(float(r[2]) for r in rows)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].strip() == "Active"})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": reasons,
+                "samples": len(rows)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def attended_pairs(T: int, B: int, k: int) -> int:
+    """Query-key pairs per head of a full causal prefill: row t sees its own
+    block up to t plus k-1 complete past blocks (all of them when fewer)."""
+    t = np.arange(T, dtype=np.int64)
+    return int(np.minimum(t + 1, (k - 1) * B + (t % B) + 1).sum())
+
+
+# ---------------------------------------------------------------------------
+# prefill workload
+# ---------------------------------------------------------------------------
+def run_prefill(w, steps, warmup, world):
+    import block_sparse_gqa_mean_b200 as msa
+    dev = torch.device("cuda")
+    T = w.ctx[0]
+    p = workloads.paging(w)
+    cache = msa.PagedKVCache.allocate(1, p.num_pages, p.max_blocks, w.hq, w.hkv, w.d, w.block,
+                                      w.torch_dtype, dev)
+    cache.page_table.copy_(p.table.to(dev))
+    cache.seq_lens.fill_(T)
+    k_new = workloads.keys(w, 0, 0, T, dev).contiguous()
+    v_new = workloads.values(w, 0, 0, T, dev).contiguous()
+    q = workloads.queries_prefill(w, 0, 0, T, dev).contiguous()
+    cu = msa.cu_seqlens([T], dev)
+    idx = torch.empty(T, w.hkv, w.top_k, dtype=torch.int32, device=dev)
+    out = torch.empty_like(q)
+    lse = torch.empty(T, w.hq, dtype=torch.float32, device=dev)
+    ws_sel = torch.empty(max(16, msa.workspace_size(msa.MSA_OP_SELECT, cache, T, T, w.top_k)),
+                         dtype=torch.uint8, device=dev)
+    ws_att = torch.empty(max(16, msa.workspace_size(msa.MSA_OP_PREFILL, cache, T, T, w.top_k)),
+                         dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev: ev[0].record(stream)
+        msa.build_block_cache(cache, k_new, v_new, cu, T)
+        if ev: ev[1].record(stream)
+        msa.select_topk(cache, q, w.top_k, cu_q=cu, max_rows_per_seq=T, block_idx=idx,
+                        workspace=ws_sel)
+        if ev: ev[2].record(stream)
+        msa.sparse_attn_prefill(cache, q, idx, cu_q=cu, max_rows_per_seq=T, out=out, lse=lse,
+                                workspace=ws_att)
+        if ev: ev[3].record(stream)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    if cache.device_status() != 0:
+        raise RuntimeError(f"device status {cache.device_status():#x}")
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    with Clocks(torch.cuda.current_device()) as clk:
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for i in range(steps):
+            step(evs[i])
+        t1.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    total_ms = t0.elapsed_time(t1)
+    k_ms = [sum(e[i].elapsed_time(e[i + 1]) for e in evs) / steps for i in range(3)]
+
+    # executed (union) tile-blocks of the tensor-core schedule, for context
+    G = w.group
+    TM = 128 // G
+    sel = idx.cpu().numpy()
+    union_blocks = 0
+    for g in range(w.hkv):
+        for t0_ in range(0, T, TM):
+            union_blocks += len(np.unique(sel[t0_:t0_ + TM, g][sel[t0_:t0_ + TM, g] >= 0]))
+
+    # end to end through the C ABI from pinned host buffers
+    hq_ = q.cpu().pin_memory()
+    hk = k_new.cpu().pin_memory()
+    hv = v_new.cpu().pin_memory()
+    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k_new), torch.empty_like(v_new)
+
+    def e2e_step():
+        dq.copy_(hq_, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        msa.build_block_cache(cache, dk, dv, cu, T)
+        msa.select_topk(cache, dq, w.top_k, cu_q=cu, max_rows_per_seq=T, block_idx=idx,
+                        workspace=ws_sel)
+        msa.sparse_attn_prefill(cache, dq, idx, cu_q=cu, max_rows_per_seq=T, out=out, lse=lse,
+                                workspace=ws_att)
+        hout.copy_(out, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        e2e_step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = a.elapsed_time(b) / steps
+    h2d = hq_.numel() * 2 + hk.numel() * 2 + hv.numel() * 2
+    d2h = hout.numel() * 2
+    status = cache.device_status()
+    if status != 0:
+        raise RuntimeError(f"device status {status:#x}")
+    return {"total_ms": total_ms, "kernel_ms": k_ms, "clocks": clk.summary(),
+            "union_blocks": union_blocks, "e2e_ms": e2e_ms, "h2d": h2d, "d2h": d2h,
+            "launches_per_step": 4}
+
+
+# ---------------------------------------------------------------------------
+# decode workloads
+# ---------------------------------------------------------------------------
+def fill_decode_cache(w, dev):
+    import block_sparse_gqa_mean_b200 as msa
+    p = workloads.paging(w)
+    cache = msa.PagedKVCache.allocate(w.batch, p.num_pages, p.max_blocks, w.hq, w.hkv, w.d,
+                                      w.block, w.torch_dtype, dev)
+    cache.page_table.copy_(p.table.to(dev))
+    lens = [0] * w.batch
+    chunk = 1 << 16
+    for b in range(w.batch):
+        for u0 in range(0, w.ctx[b], chunk):
+            u1 = min(w.ctx[b], u0 + chunk)
+            after = list(lens)
+            after[b] = u1
+            n = [after[i] - lens[i] for i in range(w.batch)]
+            cache.seq_lens.copy_(torch.tensor(after, dtype=torch.int32))
+            msa.build_block_cache(cache, workloads.keys(w, b, u0, u1, dev),
+                                  workloads.values(w, b, u0, u1, dev), msa.cu_seqlens(n, dev),
+                                  max(n))
+            lens = after
+    torch.cuda.synchronize()
+    return cache
+
+
+def decode_bytes(w, step=0):
+    """Algorithmic HBM bytes of one decode step: the centroid scan of every
+    complete past block, the K/V rows of the selected blocks (own block up to
+    the new token), q in / out, the appended K/V row and its centroid."""
+    tot = 0
+    for b in range(w.batch):
+        L = w.ctx[b] + step + 1
+        own = (L - 1) // w.block
+        cand = own
+        take = min(w.top_k - 1, cand)
+        keys = take * w.block + (L - own * w.block)
+        tot += w.hkv * (cand * w.d * 4 + keys * w.d * 2 * 2)
+        tot += 2 * w.hq * w.d * 2 + 2 * w.hkv * w.d * 2 + w.hkv * w.d * 4
+    return tot
+
+
+def run_decode(w, steps, warmup, world, flush_l2):
+    import block_sparse_gqa_mean_b200 as msa
+    dev = torch.device("cuda")
+    cache = fill_decode_cache(w, dev)
+    after = [w.ctx[b] + 1 for b in range(w.batch)]
+    cache.seq_lens.copy_(torch.tensor(after, dtype=torch.int32))
+    kn, vn = workloads.new_tokens(w, 0, dev)
+    q = workloads.queries_decode(w, 0, dev).contiguous()
+    cu = msa.cu_seqlens([1] * w.batch, dev)
+    idx = torch.empty(w.batch, w.hkv, w.top_k, dtype=torch.int32, device=dev)
+    out = torch.empty_like(q)
+    lse = torch.empty(w.batch, w.hq, dtype=torch.float32, device=dev)
+    ws_sel = torch.empty(max(16, msa.workspace_size(msa.MSA_OP_SELECT, cache, w.batch, 1, w.top_k)),
+                         dtype=torch.uint8, device=dev)
+    ws_dec = torch.empty(max(16, msa.workspace_size(msa.MSA_OP_DECODE, cache, w.batch, 1, w.top_k)),
+                         dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if flush_l2 else None
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev: ev[0].record(stream)
+        msa.build_block_cache(cache, kn, vn, cu, 1)
+        if ev: ev[1].record(stream)
+        msa.select_topk(cache, q, w.top_k, block_idx=idx, workspace=ws_sel)
+        if ev: ev[2].record(stream)
+        msa.sparse_attn_decode(cache, q, idx, out=out, lse=lse, workspace=ws_dec)
+        if ev: ev[3].record(stream)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    with Clocks(torch.cuda.current_device()) as clk:
+        for i in range(steps):
+            if flush is not None:
+                flush.fill_(i & 0xFF)
+            step(evs[i])
+        torch.cuda.synchronize()
+    barrier(world)
+    per_step = [e[0].elapsed_time(e[3]) for e in evs]
+    k_ms = [sum(e[i].elapsed_time(e[i + 1]) for e in evs) / steps for i in range(3)]
+
+    # end to end: q and the new K/V rows from pinned host memory, out back to host
+    hq_, hk, hv = q.cpu().pin_memory(), kn.cpu().pin_memory(), vn.cpu().pin_memory()
+    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(kn), torch.empty_like(vn)
+
+    def e2e_step():
+        dq.copy_(hq_, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        msa.build_block_cache(cache, dk, dv, cu, 1)
+        msa.select_topk(cache, dq, w.top_k, block_idx=idx, workspace=ws_sel)
+        msa.sparse_attn_decode(cache, dq, idx, out=out, lse=lse, workspace=ws_dec)
+        hout.copy_(out, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    e2e = []
+    for _ in range(steps):
+        if flush is not None:
+            flush.fill_(1)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        e2e_step()
+        b.record(stream)
+        e2e.append((a, b))
+    torch.cuda.synchronize()
+    e2e_ms = sum(a.elapsed_time(b) for a, b in e2e) / steps
+    status = cache.device_status()
+    if status != 0:
+        raise RuntimeError(f"device status {status:#x}")
+    return {"step_ms": sum(per_step) / steps, "kernel_ms": k_ms, "clocks": clk.summary(),
+            "e2e_ms": e2e_ms, "h2d": (hq_.numel() + hk.numel() + hv.numel()) * 2,
+            "d2h": hout.numel() * 2, "launches_per_step": 1 + 2 + 2}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle (baseline and reference arm)
+# ---------------------------------------------------------------------------
+def oracle_prefill_sample(w, rows: int):
+    """Oracle on a bounded sample: the block cache of the whole sequence plus
+    `rows` query rows spread over the sequence. Returns (rows, seconds, threads)."""
+    import oracle
+    T = w.ctx[0]
+    K = workloads.keys(w, 0, 0, T)
+    V = workloads.values(w, 0, 0, T)
+    pos = np.linspace(0, T - 1, rows).astype(np.int64)
+    Q = torch.cat([workloads.queries_prefill(w, 0, int(r), int(r) + 1) for r in pos])
+    t = time.perf_counter()
+    oracle.forward(Q, K, V, pos, w.block, w.top_k, w.softmax_scale)
+    return rows, time.perf_counter() - t, oracle.num_threads()
+
+
+def oracle_decode_sample(w, seqs: int):
+    import oracle
+    secs, n = 0.0, 0
+    for b in range(seqs):
+        L = w.ctx[b] + 1
+        K = workloads.keys(w, b, 0, L)
+        V = workloads.values(w, b, 0, L)
+        Q = workloads.queries_decode(w, 0, seqs=[b])
+        t = time.perf_counter()
+        oracle.forward(Q, K, V, np.array([L - 1]), w.block, w.top_k, w.softmax_scale)
+        secs += time.perf_counter() - t
+        n += 1
+    return n, secs, oracle.num_threads()
+
+
+# ---------------------------------------------------------------------------
+# main
+# ---------------------------------------------------------------------------
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--workload", default="prefill_bf16", choices=list(workloads.ALL))
+    ap.add_argument("--no-decode", action="store_true", help="skip the paged-decode block")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--oracle-rows", type=int, default=256)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world, rank, local = dist_setup()
+    w = workloads.ALL[args.workload]()
+    pk = peaks()
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(reference_arm(w, args)))
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py --impl native needs a CUDA device")
+    import block_sparse_gqa_mean_b200 as msa
+    msa.load_library()
+
+    res = {}
+    if w.kind == "prefill":
+        r = run_prefill(w, args.steps, args.warmup, world)
+        ms = max_over_ranks(r["total_ms"] / args.steps, world)
+        T = w.ctx[0]
+        pairs = attended_pairs(T, w.block, w.top_k) * w.hq
+        flops = 4.0 * w.d * pairs
+        attn_ms = max_over_ranks(r["kernel_ms"][2], world)
+        achieved = flops / (attn_ms * 1e-3) / 1e12
+        executed = r["union_blocks"] * 128 * w.block * w.d * 4.0
+        traffic = profile_traffic("prefill_tc_kernel", "prefill_tc.cu")
+        res.update({
+            "metric": METRIC, "value": T * world / (ms * 1e-3), "unit": "tokens/s",
+            "ms_per_step": ms,
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"],
+                         "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"],
+                         "traffic": traffic,
+                         "peak_source": f"{pk['source']} bf16 (burst cuBLAS)",
+                         "kernel": "msa_sparse_attn_prefill (plan + prefill_tc_kernel)",
+                         "algorithmic_flops_per_launch": flops,
+                         "executed_mma_flops_per_launch": executed,
+                         "executed_tflops": executed / (attn_ms * 1e-3) / 1e12},
+            "kernels_ms": {"build_block_cache": r["kernel_ms"][0], "select_topk": r["kernel_ms"][1],
+                           "sparse_attn_prefill": r["kernel_ms"][2]},
+            "e2e": {"value": T * world / (max_over_ranks(r["e2e_ms"], world) * 1e-3),
+                    "unit": "tokens/s", "h2d_bytes_per_step": r["h2d"],
+                    "d2h_bytes_per_step": r["d2h"]},
+            "gpu_launches": r["launches_per_step"] * args.steps,
+            "clocks": r["clocks"],
+            "config": {"workload": w.name, "batch": w.batch, "seq_len": T, "q_heads": w.hq,
+                       "kv_heads": w.hkv, "head_dim": w.d, "block": w.block, "top_k": w.top_k,
+                       "l2": "inputs 0.7 GB per step > 126 MB L2, no flush"},
+        })
+        if not args.no_decode and world == 1:
+            wd = workloads.paged_decode_bf16()
+            res["decode"] = decode_block(wd, args, world, pk)
+    else:
+        res.update(decode_main(w, args, world, pk))
+
+    res.update({"n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "bf16 in, fp32 accumulate" if w.dtype == "bf16" else "f32",
+                "data": "synthetic (seeded generator, planted relevant blocks)"})
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(w, args)
+    if rank == 0:
+        print(json.dumps(res))
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def decode_block(w, args, world, pk):
+    flush = w.name == "decode_1m_bf16"
+    r = run_decode(w, args.steps, args.warmup, world, flush)
+    ms = max_over_ranks(r["step_ms"], world)
+    nbytes = decode_bytes(w)
+    return {"workload": w.name, "value": w.batch * world / (ms * 1e-3), "unit": "tokens/s",
+            "ms_per_step": ms, "hbm_gbs": nbytes / (ms * 1e-3) / 1e9,
+            "roofline": {"bound": "hbm", "achieved": nbytes / (ms * 1e-3) / 1e9,
+                         "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": nbytes / (ms * 1e-3) / 1e9 / pk["hbm_gbs"],
+                         "traffic": None, "scope": "whole decode step (append+select+attention)",
+                         "algorithmic_bytes_per_step": nbytes},
+            "kernels_ms": {"build_block_cache": r["kernel_ms"][0], "select_topk": r["kernel_ms"][1],
+                           "sparse_attn_decode": r["kernel_ms"][2]},
+            "e2e": {"value": w.batch * world / (r["e2e_ms"] * 1e-3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
+            "clocks": r["clocks"], "gpu_launches": r["launches_per_step"] * args.steps,
+            "l2": "256 MB write between steps" if flush else "step reads > 126 MB L2, no flush"}
+
+
+def decode_main(w, args, world, pk):
+    d = decode_block(w, args, world, pk)
+    return {"metric": METRIC, "value": d["value"], "unit": "tokens/s", "ms_per_step": d["ms_per_step"],
+            "roofline": d["roofline"], "kernels_ms": d["kernels_ms"], "e2e": d["e2e"],
+            "clocks": d["clocks"], "gpu_launches": d["gpu_launches"],
+            "config": {"workload": w.name, "batch": w.batch, "q_heads": w.hq, "kv_heads": w.hkv,
+                       "head_dim": w.d, "block": w.block, "top_k": w.top_k,
+                       "context_mean": float(np.mean(w.ctx)), "l2": d["l2"]}}
+
+
+def cpu_baseline(w, args):
+    if w.kind == "prefill":
+        n, secs, thr = oracle_prefill_sample(w, args.oracle_rows)
+        return {"value": n / secs, "unit": "tokens/s", "cores": thr, "kind": "oracle",
+                "sample": f"{n} query rows spread over the {w.ctx[0]}-token sequence, plus the "
+                          f"block cache of the whole sequence, fp64, OpenMP"}
+    seqs = min(w.batch, 2)
+    n, secs, thr = oracle_decode_sample(w, seqs)
+    return {"value": n / secs, "unit": "tokens/s", "cores": thr, "kind": "oracle",
+            "sample": f"{n} of {w.batch} sequences' decode step (block cache of the whole "
+                      f"context + selection + attention), fp64, OpenMP"}
+
+
+def reference_arm(w, args):
+    """The CPU oracle timed as the reference arm: each step is a bounded sample."""
+    steps = []
+    for i in range(args.warmup + args.steps):
+        if w.kind == "prefill":
+            n, secs, thr = oracle_prefill_sample(w, max(8, args.oracle_rows // 4))
+        else:
+            n, secs, thr = oracle_decode_sample(w, 1)
+        if i >= args.warmup:
+            steps.append((n, secs))
+    n = sum(s[0] for s in steps)
+    secs = sum(s[1] for s in steps)
+    value = n / secs
+    sample = (f"{steps[0][0]} query rows of the {w.ctx[0]}-token prefill per step"
+              if w.kind == "prefill" else "1 sequence's decode step per step")
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * secs / len(steps), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": thr, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,284 @@
+"""Block-sparse GQA attention with a mean-pooled block cache, for B200 (sm_100a).
+
+Thin Python binding of libmsa.so (include/msa.h). It only marshals torch CUDA
+tensors into the C ABI: device pointers, host integers and the current CUDA
+stream. Every step of the computation runs in the library's CUDA kernels;
+there is no CPU or framework fallback, and importing the binding without the
+built library raises.
+
+    cache = PagedKVCache.allocate(batch=1, num_pages=..., max_blocks_per_seq=...,
+                                  num_q_heads=32, num_kv_heads=4, head_dim=128,
+                                  block_size=128, dtype=torch.bfloat16)
+    cache.page_table.copy_(table); cache.seq_lens.copy_(lens_after_append)
+    build_block_cache(cache, k_new, v_new, cu_new, max_new_per_seq)
+    idx, _ = select_topk(cache, q, top_k=16, cu_q=cu_q, max_rows_per_seq=T)
+    out, lse = sparse_attn_prefill(cache, q, idx, cu_q=cu_q, max_rows_per_seq=T)
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import math
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmsa.so")
+
+MSA_OK, MSA_ERR_INVALID_ARG, MSA_ERR_UNSUPPORTED, MSA_ERR_WORKSPACE, MSA_ERR_CUDA = range(5)
+MSA_DTYPE_BF16, MSA_DTYPE_F32 = 0, 1
+MSA_OP_SELECT, MSA_OP_PREFILL, MSA_OP_DECODE = 0, 1, 2
+MSA_DEV_BAD_PAGE, MSA_DEV_BAD_LENGTH, MSA_DEV_BAD_INDEX, MSA_DEV_TIMEOUT = 1, 2, 4, 8
+
+EXPORTS = ("msa_build_block_cache", "msa_select_topk", "msa_sparse_attn_prefill",
+           "msa_sparse_attn_decode", "msa_workspace_size", "msa_status_string", "msa_version")
+
+
+class MsaError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {status_string(status)} (status {status})")
+        self.status = status
+
+
+class _PagedKV(ctypes.Structure):
+    _fields_ = [
+        ("dtype", ctypes.c_int32),
+        ("num_q_heads", ctypes.c_int32),
+        ("num_kv_heads", ctypes.c_int32),
+        ("head_dim", ctypes.c_int32),
+        ("block_size", ctypes.c_int32),
+        ("batch", ctypes.c_int32),
+        ("num_pages", ctypes.c_int32),
+        ("max_blocks_per_seq", ctypes.c_int32),
+        ("k_pages", ctypes.c_void_p),
+        ("v_pages", ctypes.c_void_p),
+        ("centroids", ctypes.c_void_p),
+        ("page_table", ctypes.c_void_p),
+        ("seq_lens", ctypes.c_void_p),
+        ("status_word", ctypes.c_void_p),
+    ]
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libmsa.so. Raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise ImportError(f"libmsa.so not found at {path}; build it with "
+                          "`python -m block_sparse_gqa_mean_b200.build`")
+    lib = ctypes.CDLL(path)
+    P, I32, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+    KV = ctypes.POINTER(_PagedKV)
+    lib.msa_build_block_cache.argtypes = [KV, P, P, P, I32, P]
+    lib.msa_select_topk.argtypes = [KV, P, P, I32, I32, I32, P, P, P, SZ, P]
+    lib.msa_sparse_attn_prefill.argtypes = [KV, P, P, I32, I32, P, I32, ctypes.c_float, P, P, P,
+                                            SZ, P]
+    lib.msa_sparse_attn_decode.argtypes = [KV, P, P, I32, ctypes.c_float, P, P, P, SZ, P]
+    lib.msa_workspace_size.argtypes = [ctypes.c_int, KV, I32, I32, I32]
+    lib.msa_workspace_size.restype = SZ
+    lib.msa_status_string.argtypes = [ctypes.c_int]
+    lib.msa_status_string.restype = ctypes.c_char_p
+    lib.msa_version.restype = I32
+    for name in ("msa_build_block_cache", "msa_select_topk", "msa_sparse_attn_prefill",
+                 "msa_sparse_attn_decode"):
+        getattr(lib, name).restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return load_library().msa_status_string(status).decode()
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(status: int, what: str):
+    if status != MSA_OK:
+        raise MsaError(status, what)
+
+
+def _require_cuda(*ts):
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("tensors must be contiguous CUDA tensors")
+
+
+@dataclasses.dataclass
+class PagedKVCache:
+    """Caller-owned paged cache: K/V pages, fp32 centroids (block cache sharing the
+    page ids), page table, sequence lengths and the device status word."""
+    k_pages: torch.Tensor      # [num_pages, Hkv, B, d]
+    v_pages: torch.Tensor      # [num_pages, Hkv, B, d]
+    centroids: torch.Tensor    # [num_pages, Hkv, d] fp32
+    page_table: torch.Tensor   # [batch, max_blocks_per_seq] int32
+    seq_lens: torch.Tensor     # [batch] int32
+    status_word: torch.Tensor  # [4] int32 (first word used)
+    num_q_heads: int
+
+    @classmethod
+    def allocate(cls, batch: int, num_pages: int, max_blocks_per_seq: int, num_q_heads: int,
+                 num_kv_heads: int, head_dim: int, block_size: int,
+                 dtype: torch.dtype = torch.bfloat16, device="cuda") -> "PagedKVCache":
+        kp = torch.zeros(num_pages, num_kv_heads, block_size, head_dim, dtype=dtype, device=device)
+        vp = torch.zeros_like(kp)
+        cen = torch.zeros(num_pages, num_kv_heads, head_dim, dtype=torch.float32, device=device)
+        pt = torch.full((batch, max_blocks_per_seq), -1, dtype=torch.int32, device=device)
+        sl = torch.zeros(batch, dtype=torch.int32, device=device)
+        st = torch.zeros(4, dtype=torch.int32, device=device)
+        return cls(kp, vp, cen, pt, sl, st, num_q_heads)
+
+    @property
+    def num_kv_heads(self) -> int:
+        return self.k_pages.shape[1]
+
+    @property
+    def block_size(self) -> int:
+        return self.k_pages.shape[2]
+
+    @property
+    def head_dim(self) -> int:
+        return self.k_pages.shape[3]
+
+    @property
+    def batch(self) -> int:
+        return self.page_table.shape[0]
+
+    @property
+    def dtype(self) -> torch.dtype:
+        return self.k_pages.dtype
+
+    def struct(self) -> _PagedKV:
+        _require_cuda(self.k_pages, self.v_pages, self.centroids, self.page_table, self.seq_lens,
+                      self.status_word)
+        if self.k_pages.dtype == torch.bfloat16:
+            dt = MSA_DTYPE_BF16
+        elif self.k_pages.dtype == torch.float32:
+            dt = MSA_DTYPE_F32
+        else:
+            raise TypeError("K/V pages must be bf16 or fp32")
+        return _PagedKV(dt, self.num_q_heads, self.num_kv_heads, self.head_dim, self.block_size,
+                        self.batch, self.k_pages.shape[0], self.page_table.shape[1],
+                        self.k_pages.data_ptr(), self.v_pages.data_ptr(),
+                        self.centroids.data_ptr(), self.page_table.data_ptr(),
+                        self.seq_lens.data_ptr(), self.status_word.data_ptr())
+
+    def device_status(self) -> int:
+        """Read (synchronously) the device status word."""
+        return int(self.status_word[0].item()) & 0xFFFFFFFF
+
+    def clear_status(self):
+        self.status_word.zero_()
+
+
+def workspace_size(op: int, cache: PagedKVCache, num_rows: int, max_rows_per_seq: int,
+                   top_k: int) -> int:
+    kv = cache.struct()
+    return int(load_library().msa_workspace_size(op, ctypes.byref(kv), num_rows, max_rows_per_seq,
+                                                 top_k))
+
+
+def _workspace(op, cache, num_rows, max_rows, top_k, workspace):
+    need = workspace_size(op, cache, num_rows, max_rows, top_k)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=cache.k_pages.device)
+    return workspace, workspace.numel() * workspace.element_size()
+
+
+def build_block_cache(cache: PagedKVCache, k_new: torch.Tensor, v_new: torch.Tensor,
+                      cu_new: torch.Tensor, max_new_per_seq: int, stream=None) -> None:
+    """Append k_new/v_new rows (cache.seq_lens already counts them) and re-pool
+    the centroids of every touched block."""
+    lib = load_library()
+    _require_cuda(k_new, v_new, cu_new)
+    kv = cache.struct()
+    _check(lib.msa_build_block_cache(ctypes.byref(kv), _ptr(k_new), _ptr(v_new), _ptr(cu_new),
+                                     int(max_new_per_seq), _stream(stream)),
+           "msa_build_block_cache")
+
+
+def select_topk(cache: PagedKVCache, q: torch.Tensor, top_k: int,
+                cu_q: Optional[torch.Tensor] = None, max_rows_per_seq: int = 1,
+                block_idx: Optional[torch.Tensor] = None, block_score: Optional[torch.Tensor] = None,
+                want_scores: bool = False, workspace: Optional[torch.Tensor] = None,
+                stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Per-group top-k block selection. cu_q None = decode (one row per sequence)."""
+    lib = load_library()
+    _require_cuda(q, cu_q, block_idx, block_score)
+    rows = q.shape[0]
+    if block_idx is None:
+        block_idx = torch.empty(rows, cache.num_kv_heads, top_k, dtype=torch.int32, device=q.device)
+    if block_score is None and want_scores:
+        block_score = torch.empty(rows, cache.num_kv_heads, top_k, dtype=torch.float32,
+                                  device=q.device)
+    mr = 1 if cu_q is None else max_rows_per_seq
+    ws, ws_bytes = _workspace(MSA_OP_SELECT, cache, rows, mr, top_k, workspace)
+    kv = cache.struct()
+    _check(lib.msa_select_topk(ctypes.byref(kv), _ptr(q), _ptr(cu_q), rows, mr, top_k,
+                               _ptr(block_idx), _ptr(block_score), _ptr(ws), ws_bytes,
+                               _stream(stream)), "msa_select_topk")
+    return block_idx, block_score
+
+
+def sparse_attn_prefill(cache: PagedKVCache, q: torch.Tensor, block_idx: torch.Tensor,
+                        cu_q: torch.Tensor, max_rows_per_seq: int,
+                        softmax_scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
+                        lse: Optional[torch.Tensor] = None, want_lse: bool = True,
+                        workspace: Optional[torch.Tensor] = None, stream=None):
+    """Exact attention of the query rows over their selected blocks."""
+    lib = load_library()
+    _require_cuda(q, block_idx, cu_q, out, lse)
+    rows, top_k = q.shape[0], block_idx.shape[-1]
+    scale = 1.0 / math.sqrt(cache.head_dim) if softmax_scale is None else softmax_scale
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty(rows, q.shape[1], dtype=torch.float32, device=q.device)
+    ws, ws_bytes = _workspace(MSA_OP_PREFILL, cache, rows, max_rows_per_seq, top_k, workspace)
+    kv = cache.struct()
+    _check(lib.msa_sparse_attn_prefill(ctypes.byref(kv), _ptr(q), _ptr(cu_q), rows,
+                                       max_rows_per_seq, _ptr(block_idx), top_k, scale, _ptr(out),
+                                       _ptr(lse), _ptr(ws), ws_bytes, _stream(stream)),
+           "msa_sparse_attn_prefill")
+    return out, lse
+
+
+def sparse_attn_decode(cache: PagedKVCache, q: torch.Tensor, block_idx: torch.Tensor,
+                       softmax_scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
+                       lse: Optional[torch.Tensor] = None, want_lse: bool = True,
+                       workspace: Optional[torch.Tensor] = None, stream=None):
+    """Attention of one new query per sequence (at seq_lens-1) over its selected blocks."""
+    lib = load_library()
+    _require_cuda(q, block_idx, out, lse)
+    top_k = block_idx.shape[-1]
+    scale = 1.0 / math.sqrt(cache.head_dim) if softmax_scale is None else softmax_scale
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty(q.shape[0], q.shape[1], dtype=torch.float32, device=q.device)
+    ws, ws_bytes = _workspace(MSA_OP_DECODE, cache, q.shape[0], 1, top_k, workspace)
+    kv = cache.struct()
+    _check(lib.msa_sparse_attn_decode(ctypes.byref(kv), _ptr(q), _ptr(block_idx), top_k, scale,
+                                      _ptr(out), _ptr(lse), _ptr(ws), ws_bytes, _stream(stream)),
+           "msa_sparse_attn_decode")
+    return out, lse
+
+
+def cu_seqlens(lengths, device="cuda") -> torch.Tensor:
+    """[0, l0, l0+l1, ...] as int32 on `device`."""
+    c = [0]
+    for x in lengths:
+        c.append(c[-1] + int(x))
+    return torch.tensor(c, dtype=torch.int32, device=device)

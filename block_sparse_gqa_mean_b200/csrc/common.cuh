@@ -1,0 +1,66 @@
+// Shared device helpers of libmsa (internal header).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "msa.h"
+
+namespace msa {
+
+typedef __nv_bfloat16 bf16;
+
+// Bounded spin limit for every device-side wait (mbarrier polls). At a few
+// hundred ns per poll this is well above any legitimate wait and well below a
+// second, after which the kernel records MSA_DEV_TIMEOUT and unwinds.
+constexpr uint32_t kSpinLimit = 1u << 22;
+
+__device__ __forceinline__ void report(uint32_t* status, uint32_t bits) {
+  if (status) atomicOr(status, bits);
+}
+
+template <typename T>
+__device__ __forceinline__ float to_f32(T x);
+template <>
+__device__ __forceinline__ float to_f32<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ float to_f32<bf16>(bf16 x) { return __bfloat162float(x); }
+
+template <typename T>
+__device__ __forceinline__ T from_f32(float x);
+template <>
+__device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ bf16 from_f32<bf16>(float x) { return __float2bfloat16_rn(x); }
+
+// Position of query row i of sequence b: the rows are the last n_b tokens.
+__device__ __forceinline__ int row_position(int seq_len, int n_rows, int i) {
+  return seq_len - n_rows + i;
+}
+
+// ---------------------------------------------------------------------------
+// Canonical block score. Every selection kernel computes
+//   qbar[i]  = q_{h0}[i] + q_{h0+1}[i] + ... (left to right over the group's heads)
+//   score    = fma(qbar[D-1], c[D-1], ... fma(qbar[1], c[1], fma(qbar[0], c[0], 0)))
+// i.e. one fp32 fma chain in coordinate order, so a row scored by the prefill
+// kernel and the same row scored by the decode kernel give identical bits,
+// and identical centroids give identical scores (exact ties).
+// ---------------------------------------------------------------------------
+// Orderable 64-bit selection key: larger key = better (higher score, then
+// lower block index). 0 is below every real key.
+__device__ __forceinline__ uint64_t sel_key(float s, int j) {
+  if (s == 0.f) s = 0.f;  // one key for +0 and -0
+  uint32_t b = __float_as_uint(s);
+  b = (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+  return ((uint64_t)b << 32) | (uint32_t)(0x7fffffff - j);
+}
+__device__ __forceinline__ int key_block(uint64_t k) { return 0x7fffffff - (int)(uint32_t)k; }
+__device__ __forceinline__ float key_score(uint64_t k) {
+  uint32_t b = (uint32_t)(k >> 32);
+  b = (b & 0x80000000u) ? (b & 0x7fffffffu) : ~b;
+  return __uint_as_float(b);
+}
+
+}  // namespace msa

@@ -1,0 +1,220 @@
+// C-ABI entry points of libmsa: host-side validation, kernel dispatch and
+// workspace sizing. See include/msa.h for the contract of each call.
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "tma.cuh"
+
+namespace msa {
+
+// kernels (defined in the other translation units)
+cudaError_t append_pool(const msa_paged_kv_t*, const void*, const void*, const int32_t*, int,
+                        cudaStream_t);
+cudaError_t select_rows(const msa_paged_kv_t*, const void*, const int32_t*, int, int, int32_t*,
+                        float*, cudaStream_t);
+bool select_rows_supported(int top_k);
+size_t select_decode_ws(const msa_paged_kv_t*, int top_k);
+cudaError_t select_decode(const msa_paged_kv_t*, const void*, int, int32_t*, float*, void*,
+                          cudaStream_t);
+cudaError_t attn_simt(const msa_paged_kv_t*, const void*, const int32_t*, int, const int32_t*, int,
+                      float, void*, float*, cudaStream_t);
+size_t decode_ws(const msa_paged_kv_t*, int top_k, int num_sms);
+cudaError_t decode_splitk(const msa_paged_kv_t*, const void*, const int32_t*, int, float, void*,
+                          float*, void*, int, cudaStream_t);
+bool prefill_tc_supported(const msa_paged_kv_t*);
+size_t prefill_ws(const msa_paged_kv_t*, int max_rows, int top_k);
+cudaError_t prefill_tc(const msa_paged_kv_t*, const void*, const int32_t*, int, const int32_t*,
+                       int, float, void*, float*, void*, cudaStream_t);
+
+// ---------------------------------------------------------------------------
+// tensor maps (driver entry point resolved once through the runtime)
+// ---------------------------------------------------------------------------
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+bool make_tmap_bf16_2d(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                       uint32_t box_cols, uint32_t box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------------------
+// validation helpers
+// ---------------------------------------------------------------------------
+static bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+static msa_status_t check_kv(const msa_paged_kv_t* kv) {
+  if (!kv) return MSA_ERR_INVALID_ARG;
+  if (kv->dtype != MSA_DTYPE_BF16 && kv->dtype != MSA_DTYPE_F32) return MSA_ERR_UNSUPPORTED;
+  if (kv->num_q_heads <= 0 || kv->num_kv_heads <= 0 || kv->batch <= 0 || kv->num_pages <= 0 ||
+      kv->max_blocks_per_seq <= 0)
+    return MSA_ERR_INVALID_ARG;
+  if (kv->num_q_heads % kv->num_kv_heads != 0) return MSA_ERR_INVALID_ARG;
+  if (kv->num_q_heads / kv->num_kv_heads > 16) return MSA_ERR_UNSUPPORTED;
+  if (kv->head_dim != 64 && kv->head_dim != 128) return MSA_ERR_UNSUPPORTED;
+  if (kv->block_size != 64 && kv->block_size != 128) return MSA_ERR_UNSUPPORTED;
+  if ((uint64_t)kv->num_pages * kv->num_kv_heads * kv->block_size >= (1ull << 31))
+    return MSA_ERR_UNSUPPORTED;
+  if ((uint64_t)kv->max_blocks_per_seq * kv->block_size >= (1ull << 31)) return MSA_ERR_UNSUPPORTED;
+  if (!kv->k_pages || !kv->v_pages || !kv->centroids || !kv->page_table || !kv->seq_lens ||
+      !kv->status_word)
+    return MSA_ERR_INVALID_ARG;
+  if (!aligned(kv->k_pages, 16) || !aligned(kv->v_pages, 16) || !aligned(kv->centroids, 16) ||
+      !aligned(kv->page_table, 4) || !aligned(kv->seq_lens, 4) || !aligned(kv->status_word, 4))
+    return MSA_ERR_INVALID_ARG;
+  return MSA_OK;
+}
+
+static int num_sms() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+static bool use_decode_splitk(const msa_paged_kv_t* kv) {
+  return kv->dtype == MSA_DTYPE_BF16 && kv->head_dim == 128;
+}
+
+static msa_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? MSA_OK : MSA_ERR_CUDA; }
+
+}  // namespace msa
+
+using namespace msa;
+
+extern "C" {
+
+int32_t msa_version(void) { return 1000; }
+
+const char* msa_status_string(msa_status_t s) {
+  switch (s) {
+    case MSA_OK: return "ok";
+    case MSA_ERR_INVALID_ARG: return "invalid argument";
+    case MSA_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case MSA_ERR_WORKSPACE: return "workspace too small";
+    case MSA_ERR_CUDA: return "CUDA launch error";
+  }
+  return "unknown status";
+}
+
+size_t msa_workspace_size(msa_op_t op, const msa_paged_kv_t* kv, int32_t num_rows,
+                          int32_t max_rows_per_seq, int32_t top_k) {
+  (void)num_rows;
+  if (check_kv(kv) != MSA_OK || top_k < 1 || top_k > 256) return 0;
+  switch (op) {
+    case MSA_OP_SELECT:
+      return max_rows_per_seq <= 1 ? select_decode_ws(kv, top_k) : 0;
+    case MSA_OP_PREFILL:
+      return prefill_tc_supported(kv) && max_rows_per_seq > 0
+                 ? prefill_ws(kv, max_rows_per_seq, top_k) : 0;
+    case MSA_OP_DECODE:
+      return use_decode_splitk(kv) ? decode_ws(kv, top_k, num_sms()) : 0;
+  }
+  return 0;
+}
+
+msa_status_t msa_build_block_cache(const msa_paged_kv_t* kv, const void* k_new, const void* v_new,
+                                   const int32_t* cu_new, int32_t max_new_per_seq,
+                                   msa_stream_t stream) {
+  msa_status_t s = check_kv(kv);
+  if (s != MSA_OK) return s;
+  if (max_new_per_seq < 0) return MSA_ERR_INVALID_ARG;
+  if (max_new_per_seq == 0) return MSA_OK;
+  if (!k_new || !v_new || !cu_new || !aligned(k_new, 16) || !aligned(v_new, 16) ||
+      !aligned(cu_new, 4))
+    return MSA_ERR_INVALID_ARG;
+  return from_cuda(append_pool(kv, k_new, v_new, cu_new, max_new_per_seq, (cudaStream_t)stream));
+}
+
+msa_status_t msa_select_topk(const msa_paged_kv_t* kv, const void* q, const int32_t* cu_q,
+                             int32_t num_rows, int32_t max_rows_per_seq, int32_t top_k,
+                             int32_t* block_idx, float* block_score, void* workspace,
+                             size_t workspace_bytes, msa_stream_t stream) {
+  msa_status_t s = check_kv(kv);
+  if (s != MSA_OK) return s;
+  if (top_k < 1 || top_k > 256) return MSA_ERR_UNSUPPORTED;
+  if (num_rows < 0 || max_rows_per_seq < 0) return MSA_ERR_INVALID_ARG;
+  if (num_rows == 0) return MSA_OK;
+  if (!q || !block_idx || !aligned(q, 16) || !aligned(block_idx, 4) ||
+      (block_score && !aligned(block_score, 4)))
+    return MSA_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (!cu_q) {
+    if (num_rows != kv->batch) return MSA_ERR_INVALID_ARG;
+    const size_t need = select_decode_ws(kv, top_k);
+    if (workspace_bytes < need || (need && (!workspace || !aligned(workspace, 16))))
+      return MSA_ERR_WORKSPACE;
+    return from_cuda(select_decode(kv, q, top_k, block_idx, block_score, workspace, st));
+  }
+  if (!aligned(cu_q, 4) || max_rows_per_seq < 1) return MSA_ERR_INVALID_ARG;
+  if (!select_rows_supported(top_k)) return MSA_ERR_UNSUPPORTED;
+  return from_cuda(select_rows(kv, q, cu_q, max_rows_per_seq, top_k, block_idx, block_score, st));
+}
+
+msa_status_t msa_sparse_attn_prefill(const msa_paged_kv_t* kv, const void* q, const int32_t* cu_q,
+                                     int32_t num_rows, int32_t max_rows_per_seq,
+                                     const int32_t* block_idx, int32_t top_k, float softmax_scale,
+                                     void* out, float* lse, void* workspace,
+                                     size_t workspace_bytes, msa_stream_t stream) {
+  msa_status_t s = check_kv(kv);
+  if (s != MSA_OK) return s;
+  if (top_k < 1 || top_k > 256) return MSA_ERR_UNSUPPORTED;
+  if (num_rows < 0 || max_rows_per_seq < 0) return MSA_ERR_INVALID_ARG;
+  if (num_rows == 0) return MSA_OK;
+  if (!q || !cu_q || !block_idx || !out || !aligned(q, 16) || !aligned(out, 16) ||
+      !aligned(cu_q, 4) || !aligned(block_idx, 4) || (lse && !aligned(lse, 4)) ||
+      max_rows_per_seq < 1 || !(softmax_scale > 0.f))
+    return MSA_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (prefill_tc_supported(kv)) {
+    const size_t need = prefill_ws(kv, max_rows_per_seq, top_k);
+    if (workspace_bytes < need || !workspace || !aligned(workspace, 16)) return MSA_ERR_WORKSPACE;
+    return from_cuda(prefill_tc(kv, q, cu_q, max_rows_per_seq, block_idx, top_k, softmax_scale, out,
+                                lse, workspace, st));
+  }
+  return from_cuda(attn_simt(kv, q, cu_q, max_rows_per_seq, block_idx, top_k, softmax_scale, out,
+                             lse, st));
+}
+
+msa_status_t msa_sparse_attn_decode(const msa_paged_kv_t* kv, const void* q,
+                                    const int32_t* block_idx, int32_t top_k, float softmax_scale,
+                                    void* out, float* lse, void* workspace, size_t workspace_bytes,
+                                    msa_stream_t stream) {
+  msa_status_t s = check_kv(kv);
+  if (s != MSA_OK) return s;
+  if (top_k < 1 || top_k > 256) return MSA_ERR_UNSUPPORTED;
+  if (!q || !block_idx || !out || !aligned(q, 16) || !aligned(out, 16) || !aligned(block_idx, 4) ||
+      (lse && !aligned(lse, 4)) || !(softmax_scale > 0.f))
+    return MSA_ERR_INVALID_ARG;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (use_decode_splitk(kv)) {
+    const int sms = num_sms();
+    const size_t need = decode_ws(kv, top_k, sms);
+    if (workspace_bytes < need || !workspace || !aligned(workspace, 16)) return MSA_ERR_WORKSPACE;
+    return from_cuda(
+        decode_splitk(kv, q, block_idx, top_k, softmax_scale, out, lse, workspace, sms, st));
+  }
+  return from_cuda(attn_simt(kv, q, nullptr, 1, block_idx, top_k, softmax_scale, out, lse, st));
+}
+
+}  // extern "C"

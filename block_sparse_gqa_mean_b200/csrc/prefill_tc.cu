@@ -1,0 +1,575 @@
+// Sparse prefill attention on the 5th-generation tensor cores (tcgen05, TMEM).
+//
+// "MiniMax Sparse Attention" (staik.se), method and results paragraphs: exact
+// blockwise sparse attention over the selected blocks, made fast by keeping
+// the tensor cores busy; "Gated Sparse Attention: An Architectural Evolution
+// for Long-Context LLMs", section 4: sparse patterns are mapped onto dense
+// block matrix operations and the kernels skip the work that is masked out.
+//
+// Work unit: a query tile of TM = 128 / G consecutive tokens of one sequence
+// and one KV group, i.e. 128 query rows (token-major, the group's G heads per
+// token). The tile's tokens select their blocks independently, so the tile
+// walks the UNION of their selections (built by prefill_plan_kernel, ascending,
+// each entry carrying a bit per token that selected it). Per union block the
+// CTA computes S = Q K^T for all 128 rows on the tensor cores and the softmax
+// gives zero weight to rows whose token did not select the block.
+//
+// CTA layout (192 threads): warp 0 issues TMA loads of K and V tiles (two
+// 64-column boxes each, 128-byte swizzle, no multicast) into a 3-stage ring;
+// warp 1 owns the TMEM allocation and issues tcgen05.mma from one thread;
+// warps 2..5 are the softmax warps, one TMEM lane (query row) per thread.
+// TMEM columns: Q (bf16, A operand) | P (bf16, A operand) | S0 | S1 | O (fp32).
+//   S = Q K^T : M=128, N=B, K=128, A = Q from TMEM, B = K tile (K-major SW128)
+//   O += P V  : M=128, N=128, K=B, A = P from TMEM, B = V tile (MN-major SW128)
+// S is double-buffered so the tensor cores compute S for block e+1 while the
+// softmax warps exponentiate block e. The online softmax rescales O in TMEM
+// only when a row's running max grows.
+#include "tma.cuh"
+
+namespace msa {
+
+namespace {
+
+constexpr int kD = 128;
+constexpr float kLog2e = 1.4426950408889634f;
+
+// TMEM column map (512 columns allocated)
+constexpr uint32_t kColQ = 0;     // 64 columns: 128 bf16 per row
+constexpr uint32_t kColP = 64;    // 64 columns: up to 128 bf16 per row
+constexpr uint32_t kColS = 128;   // two 128-column fp32 buffers
+constexpr uint32_t kColO = 384;   // 128 columns fp32
+
+// ---- tcgen05 wrappers ------------------------------------------------------
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// A from TMEM, B from shared memory (descriptor), D in TMEM.
+__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n"
+      " .reg .pred p;\n"
+      " setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %5, %5, %5}, p;\n"
+      "}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0u));
+}
+
+__device__ __forceinline__ void tc_commit(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// 32 lanes x 32 consecutive 32-bit columns: thread i of the warp gets lane i.
+__device__ __forceinline__ void tc_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
+      "%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+
+__device__ __forceinline__ void tc_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
+      "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
+      "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+
+// Shared-memory matrix descriptor, 128-byte swizzle (sm_100 layout: start
+// address, leading and stride byte offsets in 16-byte units, version 1).
+__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+
+// Instruction descriptor, kind::f16: bf16 A and B, fp32 D, M x N.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) |
+         ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------
+// Planning: union of each tile's selections, ascending, with token bitmasks.
+// ---------------------------------------------------------------------------
+constexpr int kPlanWindow = 4096;
+
+__global__ void __launch_bounds__(128) prefill_plan_kernel(
+    const int32_t* __restrict__ cu_q, const int32_t* __restrict__ seq_lens,
+    const int32_t* __restrict__ block_idx, uint32_t* status, int hkv, int B, int max_blocks,
+    int top_k, int TM, int tiles_per_seq, int ecap, int2* __restrict__ entries,
+    int* __restrict__ counts) {
+  __shared__ uint32_t bm[kPlanWindow];
+  __shared__ int warp_tot[4];
+  __shared__ int s_base;
+  const int tile = blockIdx.x;
+  const int g = tile % hkv;
+  const int tt = (tile / hkv) % tiles_per_seq;
+  const int b = tile / (hkv * tiles_per_seq);
+  const int tid = threadIdx.x, lane = tid % 32, warp = tid / 32;
+  const int row0 = cu_q[b];
+  const int n_rows = cu_q[b + 1] - row0;
+  const int r_lo = tt * TM;
+  if (r_lo >= n_rows) {
+    if (tid == 0) counts[tile] = 0;
+    return;
+  }
+  const int nr = min(TM, n_rows - r_lo);
+  const int L = seq_lens[b];
+  if (n_rows > L || L > max_blocks * B) {
+    if (tid == 0) {
+      counts[tile] = 0;
+      report(status, MSA_DEV_BAD_LENGTH);
+    }
+    return;
+  }
+  const int t_first = L - n_rows + r_lo;
+  const int own_max = (t_first + nr - 1) / B;
+  const int R = own_max + 1;
+  int2* out = entries + (size_t)tile * ecap;
+  if (tid == 0) s_base = 0;
+  for (int w0 = 0; w0 < R; w0 += kPlanWindow) {
+    const int W = min(kPlanWindow, R - w0);
+    for (int i = tid; i < W; i += 128) bm[i] = 0u;
+    __syncthreads();
+    for (int it = tid; it < nr * top_k; it += 128) {
+      const int i = it / top_k, s = it % top_k;
+      const int j = block_idx[((size_t)(row0 + r_lo + i) * hkv + g) * top_k + s];
+      if (j < 0) continue;
+      const int own_i = (t_first + i) / B;
+      if (j > own_i) {
+        report(status, MSA_DEV_BAD_INDEX);
+        continue;
+      }
+      if (j >= w0 && j < w0 + W) atomicOr(&bm[j - w0], 1u << i);
+    }
+    __syncthreads();
+    // compaction: thread tid scans words [tid*per, (tid+1)*per)
+    const int per = (W + 127) / 128;
+    const int a0 = min(W, tid * per), a1 = min(W, a0 + per);
+    int cnt = 0;
+    for (int a = a0; a < a1; ++a) cnt += bm[a] != 0u;
+    int incl = cnt;
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    if (lane == 31) warp_tot[warp] = incl;
+    __syncthreads();
+    int off = s_base + incl - cnt;
+    for (int w = 0; w < warp; ++w) off += warp_tot[w];
+    for (int a = a0; a < a1; ++a)
+      if (bm[a] != 0u) out[off++] = make_int2(w0 + a, (int)bm[a]);
+    __syncthreads();
+    if (tid == 0) s_base += warp_tot[0] + warp_tot[1] + warp_tot[2] + warp_tot[3];
+    __syncthreads();
+  }
+  if (tid == 0) counts[tile] = s_base;
+}
+
+// ---------------------------------------------------------------------------
+// Attention
+// ---------------------------------------------------------------------------
+template <int B, int G>
+__global__ void __launch_bounds__(192, 1) prefill_tc_kernel(
+    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+    const bf16* __restrict__ q, const int32_t* __restrict__ cu_q,
+    const int32_t* __restrict__ page_table, const int32_t* __restrict__ seq_lens, uint32_t* status,
+    int hq, int hkv, int num_pages, int max_blocks, int tiles_per_seq, int ecap,
+    const int2* __restrict__ entries, const int* __restrict__ counts, float scale_log2,
+    bf16* __restrict__ out, float* __restrict__ lse) {
+  constexpr int TM = 128 / G;            // tokens per tile
+  constexpr int NST = (B == 128) ? 3 : 4;
+  constexpr int TILE = B * kD * 2;       // bytes of a K (or V) tile
+  constexpr int STAGE = 2 * TILE;
+  constexpr uint32_t IDESC_S = idesc_bf16(128, B, false);
+  constexpr uint32_t IDESC_O = idesc_bf16(128, kD, true);
+
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  __shared__ __align__(8) uint64_t kv_full[NST], kv_empty[NST];
+  __shared__ __align__(8) uint64_t s_full[2], s_free[2], p_full, o_done, q_ready, fin;
+  __shared__ uint32_t s_tmem;
+  __shared__ volatile int s_abort;
+
+  const int tile = blockIdx.x;
+  const int g = tile % hkv;
+  const int tt = (tile / hkv) % tiles_per_seq;
+  const int b = tile / (hkv * tiles_per_seq);
+  const int n_e = counts[tile];
+  if (n_e == 0) return;  // empty tile (ragged batch) - uniform exit before any sync
+  const int2* ent = entries + (size_t)tile * ecap;
+  const int row0 = cu_q[b];
+  const int n_rows = cu_q[b + 1] - row0;
+  const int r_lo = tt * TM;
+  const int nr = min(TM, n_rows - r_lo);
+  const int L = seq_lens[b];
+  const int t_first = L - n_rows + r_lo;
+
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  if (tid == 0) {
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&s_full[s], 1);
+      mbar_init(&s_free[s], 128);
+    }
+    mbar_init(&p_full, 128);
+    mbar_init(&o_done, 1);
+    mbar_init(&q_ready, 128);
+    mbar_init(&fin, 1);
+    s_abort = 0;
+    mbar_fence_init();
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(
+                     smem_u32(&s_tmem))
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_tmem;
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      int issued = 0;
+      for (int e = 0; e < n_e && !s_abort; ++e) {
+        const int st = e % NST;
+        if (!mbar_wait(&kv_empty[st], ((e / NST) & 1) ^ 1)) {
+          report(status, MSA_DEV_TIMEOUT);
+          s_abort = 1;
+          break;
+        }
+        const int j = ent[e].x;
+        int pg = page_table[(size_t)b * max_blocks + j];
+        if (pg < 0 || pg >= num_pages) {
+          report(status, MSA_DEV_BAD_PAGE);
+          pg = 0;  // keep the pipeline in step; the result of this tile is unspecified
+        }
+        const int y = (pg * hkv + g) * B;
+        unsigned char* kt = smem + st * STAGE;
+        mbar_expect_tx(&kv_full[st], STAGE);
+        tma_load_2d(kt, &tm_k, &kv_full[st], 0, y);
+        tma_load_2d(kt + TILE / 2, &tm_k, &kv_full[st], 64, y);
+        tma_load_2d(kt + TILE, &tm_v, &kv_full[st], 0, y);
+        tma_load_2d(kt + TILE + TILE / 2, &tm_v, &kv_full[st], 64, y);
+        ++issued;
+      }
+      // every copy issued must have landed before the CTA may exit (bounded)
+      for (int e = max(0, issued - NST); e < issued; ++e)
+        if (!mbar_wait(&kv_full[e % NST], (e / NST) & 1)) report(status, MSA_DEV_TIMEOUT);
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      bool ok = mbar_wait(&q_ready, 0);
+      tc_fence_after();
+      auto issue_s = [&](int e) -> bool {
+        const int st = e % NST, sb = e & 1;
+        if (!mbar_wait(&kv_full[st], (e / NST) & 1)) return false;
+        if (!mbar_wait(&s_free[sb], ((e >> 1) & 1) ^ 1)) return false;
+        tc_fence_after();
+        const uint32_t kt = smem_u32(smem + st * STAGE);
+#pragma unroll
+        for (int ks = 0; ks < kD / 16; ++ks) {
+          const uint32_t addr = kt + (uint32_t)(ks >> 2) * (uint32_t)(TILE / 2) + (uint32_t)(ks & 3) * 32u;
+          tc_mma_ts(tmem + kColS + sb * 128, tmem + kColQ + ks * 8, sdesc_sw128(addr, 16, 1024),
+                    IDESC_S, ks > 0);
+        }
+        tc_commit(&s_full[sb]);
+        return true;
+      };
+      if (ok) ok = issue_s(0);
+      for (int e = 0; e < n_e && ok && !s_abort; ++e) {
+        if (e + 1 < n_e) ok = issue_s(e + 1);
+        if (!ok) break;
+        if (!mbar_wait(&p_full, e & 1)) { ok = false; break; }
+        tc_fence_after();
+        const int st = e % NST;
+        const uint32_t vt = smem_u32(smem + st * STAGE + TILE);
+#pragma unroll
+        for (int kk = 0; kk < B / 16; ++kk) {
+          tc_mma_ts(tmem + kColO, tmem + kColP + kk * 8,
+                    sdesc_sw128(vt + (uint32_t)kk * 2048u, (uint32_t)(TILE / 2), 1024), IDESC_O,
+                    (e > 0 || kk > 0) ? 1u : 0u);
+        }
+        tc_commit(&o_done);
+        tc_commit(&kv_empty[st]);
+      }
+      if (!ok) {
+        report(status, MSA_DEV_TIMEOUT);
+        s_abort = 1;
+      }
+      // all MMAs issued by this thread complete before TMEM is released (bounded)
+      tc_commit(&fin);
+      if (!mbar_wait(&fin, 0)) report(status, MSA_DEV_TIMEOUT);
+    }
+  } else {
+    // ---------------- softmax warps ----------------
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;           // query row of this thread == TMEM lane
+    const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+    const int ti = r / G, h = r % G;             // token within the tile, head within the group
+    const bool row_ok = ti < nr;
+    const int t = t_first + ti;                   // position of this row's token
+    // Q row -> TMEM (bf16 pairs as 32-bit columns)
+    {
+      uint32_t qv[32];
+      const uint4* src = reinterpret_cast<const uint4*>(
+          q + ((size_t)(row0 + r_lo + ti) * hq + (size_t)g * G + h) * kD);
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          uint4 v = row_ok ? src[half * 8 + c] : make_uint4(0u, 0u, 0u, 0u);
+          qv[4 * c + 0] = v.x;
+          qv[4 * c + 1] = v.y;
+          qv[4 * c + 2] = v.z;
+          qv[4 * c + 3] = v.w;
+        }
+        tc_st32(lane_base + kColQ + half * 32, qv);
+      }
+      tc_wait_st();
+      tc_fence_before();
+      mbar_arrive(&q_ready);
+    }
+    float m = -INFINITY, l = 0.f;
+    for (int e = 0; e < n_e; ++e) {
+      if (__any_sync(0xffffffffu, s_abort != 0)) break;
+      const int sb = e & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[sb], (e >> 1) & 1))) {
+        report(status, MSA_DEV_TIMEOUT);
+        s_abort = 1;
+        break;
+      }
+      tc_fence_after();
+      float s[B];
+#pragma unroll
+      for (int c = 0; c < B / 32; ++c) {
+        uint32_t v[32];
+        tc_ld32(lane_base + kColS + sb * 128 + c * 32, v);
+        tc_wait_ld();
+#pragma unroll
+        for (int x = 0; x < 32; ++x) s[c * 32 + x] = __uint_as_float(v[x]);
+      }
+      tc_fence_before();
+      mbar_arrive(&s_free[sb]);
+
+      const int2 en = ent[e];
+      const int j = en.x;
+      const bool sel = row_ok && ((en.y >> ti) & 1);
+      float mx = -INFINITY;
+      if (sel) {
+        const int kmax = t - j * B;  // visible keys: index <= kmax
+#pragma unroll
+        for (int c = 0; c < B; ++c) {
+          s[c] = (c <= kmax) ? s[c] * scale_log2 : -INFINITY;
+          mx = fmaxf(mx, s[c]);
+        }
+      }
+      const float m_new = fmaxf(m, mx);
+      const bool rescale = sel && (m != -INFINITY) && (m_new > m);
+      const float alpha = rescale ? fast_exp2(m - m_new) : 1.f;
+      float rs = 0.f;
+      uint32_t pk[B / 2];
+      if (sel) {
+#pragma unroll
+        for (int c = 0; c < B; c += 2) {
+          // l sums the same bf16-rounded weights the P*V product uses, so the
+          // output is an exact convex combination of the rounded weights
+          const uint32_t pp = pack_bf16(fast_exp2(s[c] - m_new), fast_exp2(s[c + 1] - m_new));
+          rs += __uint_as_float(pp << 16) + __uint_as_float(pp & 0xffff0000u);
+          pk[c / 2] = pp;
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < B / 2; ++c) pk[c] = 0u;
+      }
+      // previous P*V must be complete before P is overwritten or O rescaled
+      if (e > 0) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&o_done, (e - 1) & 1))) {
+          report(status, MSA_DEV_TIMEOUT);
+          s_abort = 1;
+          break;
+        }
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+          for (int c = 0; c < kD / 32; ++c) {
+            uint32_t v[32];
+            tc_ld32(lane_base + kColO + c * 32, v);
+            tc_wait_ld();
+#pragma unroll
+            for (int x = 0; x < 32; ++x) v[x] = __float_as_uint(__uint_as_float(v[x]) * alpha);
+            tc_st32(lane_base + kColO + c * 32, v);
+          }
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < B / 64; ++c) {
+        uint32_t v[32];
+#pragma unroll
+        for (int x = 0; x < 32; ++x) v[x] = pk[c * 32 + x];
+        tc_st32(lane_base + kColP + c * 32, v);
+      }
+      tc_wait_st();
+      tc_fence_before();
+      mbar_arrive(&p_full);
+      if (sel) {
+        l = l * alpha + rs;
+        m = m_new;
+      }
+    }
+    // epilogue: O / l -> bf16
+    const bool go = !__any_sync(0xffffffffu, s_abort != 0);
+    if (go && __all_sync(0xffffffffu, mbar_wait(&o_done, (n_e - 1) & 1))) {
+      tc_fence_after();
+      const float inv = (l > 0.f) ? 1.f / l : 0.f;
+      uint4* dst = reinterpret_cast<uint4*>(
+          out + ((size_t)(row0 + r_lo + ti) * hq + (size_t)g * G + h) * kD);
+#pragma unroll
+      for (int c = 0; c < kD / 32; ++c) {
+        uint32_t v[32];
+        tc_ld32(lane_base + kColO + c * 32, v);
+        tc_wait_ld();
+        if (row_ok) {
+#pragma unroll
+          for (int x = 0; x < 32; x += 8) {
+            uint4 w;
+            w.x = pack_bf16(__uint_as_float(v[x]) * inv, __uint_as_float(v[x + 1]) * inv);
+            w.y = pack_bf16(__uint_as_float(v[x + 2]) * inv, __uint_as_float(v[x + 3]) * inv);
+            w.z = pack_bf16(__uint_as_float(v[x + 4]) * inv, __uint_as_float(v[x + 5]) * inv);
+            w.w = pack_bf16(__uint_as_float(v[x + 6]) * inv, __uint_as_float(v[x + 7]) * inv);
+            dst[(c * 32 + x) / 8] = w;
+          }
+        }
+      }
+      if (row_ok && lse)
+        lse[(size_t)(row0 + r_lo + ti) * hq + (size_t)g * G + h] =
+            (l > 0.f) ? (m + log2f(l)) * 0.6931471805599453f : -INFINITY;
+    } else if (go) {
+      report(status, MSA_DEV_TIMEOUT);
+      s_abort = 1;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem) : "memory");
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+int prefill_tile_tokens(int G) { return 128 / G; }
+
+static int plan_tiles(const msa_paged_kv_t* kv, int max_rows, int* tps) {
+  const int TM = 128 / (kv->num_q_heads / kv->num_kv_heads);
+  *tps = (max_rows + TM - 1) / TM;
+  return kv->batch * (*tps) * kv->num_kv_heads;
+}
+
+size_t prefill_ws(const msa_paged_kv_t* kv, int max_rows, int top_k) {
+  int tps;
+  const size_t tiles = plan_tiles(kv, max_rows, &tps);
+  const int TM = 128 / (kv->num_q_heads / kv->num_kv_heads);
+  const size_t ecap = (size_t)TM * top_k;
+  return tiles * ecap * sizeof(int2) + tiles * sizeof(int) + 256;
+}
+
+bool prefill_tc_supported(const msa_paged_kv_t* kv) {
+  const int G = kv->num_q_heads / kv->num_kv_heads;
+  return kv->dtype == MSA_DTYPE_BF16 && kv->head_dim == 128 && (G == 8 || G == 16) &&
+         (kv->block_size == 64 || kv->block_size == 128);
+}
+
+template <int B, int G>
+static cudaError_t launch_tc(const msa_paged_kv_t* kv, const CUtensorMap& tk, const CUtensorMap& tv,
+                             const void* q, const int32_t* cu_q, int tiles, int tps, int ecap,
+                             const int2* entries, const int* counts, float sl2, void* out,
+                             float* lse, cudaStream_t st) {
+  constexpr int NST = (B == 128) ? 3 : 4;
+  const size_t smem = (size_t)NST * 2 * B * kD * 2 + 1024;
+  auto kern = prefill_tc_kernel<B, G>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  kern<<<tiles, 192, smem, st>>>(tk, tv, (const bf16*)q, cu_q, kv->page_table, kv->seq_lens,
+                                 kv->status_word, kv->num_q_heads, kv->num_kv_heads, kv->num_pages,
+                                 kv->max_blocks_per_seq, tps, ecap, entries, counts, sl2,
+                                 (bf16*)out, lse);
+  return cudaGetLastError();
+}
+
+cudaError_t prefill_tc(const msa_paged_kv_t* kv, const void* q, const int32_t* cu_q, int max_rows,
+                       const int32_t* idx, int top_k, float scale, void* out, float* lse, void* ws,
+                       cudaStream_t st) {
+  const int G = kv->num_q_heads / kv->num_kv_heads, B = kv->block_size;
+  const int TM = 128 / G;
+  int tps;
+  const int tiles = plan_tiles(kv, max_rows, &tps);
+  const int ecap = TM * top_k;
+  int2* entries = (int2*)ws;
+  int* counts = (int*)(entries + (size_t)tiles * ecap);
+  prefill_plan_kernel<<<tiles, 128, 0, st>>>(cu_q, kv->seq_lens, idx, kv->status_word,
+                                             kv->num_kv_heads, B, kv->max_blocks_per_seq, top_k,
+                                             TM, tps, ecap, entries, counts);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  CUtensorMap tk, tv;
+  const uint64_t rows = (uint64_t)kv->num_pages * kv->num_kv_heads * B;
+  if (!make_tmap_bf16_2d(&tk, kv->k_pages, rows, kD, 64, B) ||
+      !make_tmap_bf16_2d(&tv, kv->v_pages, rows, kD, 64, B))
+    return cudaErrorInvalidValue;
+  const float sl2 = scale * kLog2e;
+  if (B == 128)
+    return G == 8 ? launch_tc<128, 8>(kv, tk, tv, q, cu_q, tiles, tps, ecap, entries, counts, sl2, out, lse, st)
+                  : launch_tc<128, 16>(kv, tk, tv, q, cu_q, tiles, tps, ecap, entries, counts, sl2, out, lse, st);
+  return G == 8 ? launch_tc<64, 8>(kv, tk, tv, q, cu_q, tiles, tps, ecap, entries, counts, sl2, out, lse, st)
+                : launch_tc<64, 16>(kv, tk, tv, q, cu_q, tiles, tps, ecap, entries, counts, sl2, out, lse, st);
+}
+
+}  // namespace msa

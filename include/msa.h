@@ -1,0 +1,225 @@
+/*
+ * msa.h - C ABI of the block-sparse GQA attention library (libmsa.so).
+ *
+ * The library implements MoBA-style block-sparse attention over a paged KV
+ * cache on NVIDIA B200 (sm_100a):
+ *
+ *   1. the keys of each block are mean-pooled into an fp32 centroid kept in a
+ *      block cache that is indexed by the same page ids as the K/V cache
+ *      ("Art of Focus: Ling 2.0 ...", section "Summarizing the Breakthrough":
+ *      blocks are aggregated into representations stored in a page-aware
+ *      block cache that shares the KV cache's indexing);
+ *   2. every query row scores the complete past blocks with its GQA group's
+ *      summed query and keeps its own block plus the best k-1 others, without
+ *      exponentials, ties to the lower block index ("MiniMax Sparse Attention",
+ *      method and results paragraphs: per-GQA-group top-k over KV blocks,
+ *      exp-free selection);
+ *   3. exact causal attention softmax(q k^T * scale) v runs over the tokens of
+ *      the selected blocks only ("MiniMax Sparse Attention", method paragraph;
+ *      "Sparse Attention + Linear Backbones", section 5.5).
+ *
+ * Conventions for every entry point
+ * ---------------------------------
+ *  - All tensor arguments are DEVICE pointers owned by the caller; the library
+ *    never allocates, frees or synchronises, and keeps no mutable global state
+ *    (entry points may be called from several host threads on different
+ *    streams). Every call is asynchronous on `stream`.
+ *  - Host-side validation runs before any launch. It returns
+ *    MSA_ERR_INVALID_ARG for null or misaligned pointers (16-byte alignment is
+ *    required for every tensor) and inconsistent sizes, MSA_ERR_UNSUPPORTED
+ *    for shapes outside the supported set, MSA_ERR_WORKSPACE when the
+ *    workspace is smaller than msa_workspace_size() asks for, and MSA_ERR_CUDA
+ *    when a launch fails. Nothing is launched on an error return.
+ *  - Kernels that find bad device-side data (a page id outside
+ *    [0, num_pages), a length beyond the cache's capacity, a block index out of
+ *    range) set bits of *kv->status_word (MSA_DEV_* below) and skip that unit
+ *    of work; its outputs are then unspecified. They never trap. The caller
+ *    reads the status word after synchronising and clears it when it wishes.
+ *  - Supported shapes: head_dim 64 or 128; block_size 64 or 128;
+ *    G = num_q_heads / num_kv_heads an integer in 1..16; 1 <= top_k <= 256.
+ *    bf16 attention needs head_dim 128; bf16 prefill attention needs G 8 or 16.
+ *
+ * Memory layout (all row-major)
+ *  - K/V pages       : [num_pages][num_kv_heads][block_size][head_dim], dtype
+ *  - centroids       : [num_pages][num_kv_heads][head_dim] fp32, page id as index
+ *  - page_table      : [batch][max_blocks_per_seq] int32, logical block -> page
+ *  - seq_lens        : [batch] int32, tokens in each sequence (after appends)
+ *  - queries / out   : [rows][num_q_heads][head_dim], dtype
+ *  - block_idx       : [rows][num_kv_heads][top_k] int32
+ *  Query head h belongs to KV head floor(h / G).
+ */
+#ifndef MSA_H_
+#define MSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st* msa_stream_t;
+
+typedef enum msa_status {
+  MSA_OK = 0,
+  MSA_ERR_INVALID_ARG = 1,
+  MSA_ERR_UNSUPPORTED = 2,
+  MSA_ERR_WORKSPACE = 3,
+  MSA_ERR_CUDA = 4
+} msa_status_t;
+
+typedef enum msa_dtype { MSA_DTYPE_BF16 = 0, MSA_DTYPE_F32 = 1 } msa_dtype_t;
+
+/* Bits set in *status_word by kernels that meet bad device-side data. */
+#define MSA_DEV_BAD_PAGE 0x1u   /* page id outside [0, num_pages)                   */
+#define MSA_DEV_BAD_LENGTH 0x2u /* length beyond capacity, or rows beyond seq_len   */
+#define MSA_DEV_BAD_INDEX 0x4u  /* block index outside [0, own block] or unsorted   */
+#define MSA_DEV_TIMEOUT 0x8u    /* a bounded device-side wait gave up               */
+
+/* The paged cache, passed by pointer. Host integers size the grids, so no
+ * entry point reads device memory on the host. */
+typedef struct msa_paged_kv {
+  int32_t dtype;              /* msa_dtype_t of K/V pages, queries and outputs     */
+  int32_t num_q_heads;
+  int32_t num_kv_heads;
+  int32_t head_dim;
+  int32_t block_size;         /* tokens per block == tokens per page              */
+  int32_t batch;
+  int32_t num_pages;
+  int32_t max_blocks_per_seq; /* columns of page_table                            */
+  void* k_pages;              /* device, see layout above                         */
+  void* v_pages;              /* device                                           */
+  float* centroids;           /* device, fp32                                     */
+  const int32_t* page_table;  /* device                                           */
+  const int32_t* seq_lens;    /* device                                           */
+  uint32_t* status_word;      /* device, one word                                 */
+} msa_paged_kv_t;
+
+typedef enum msa_op {
+  MSA_OP_SELECT = 0,
+  MSA_OP_PREFILL = 1,
+  MSA_OP_DECODE = 2
+} msa_op_t;
+
+/*
+ * msa_build_block_cache - append tokens to the paged cache and re-pool the
+ * centroids of every block they touch.
+ *
+ * Follows "Art of Focus: Ling 2.0 ...", "Summarizing the Breakthrough": during
+ * prefill the tokens are aggregated into block representations stored in the
+ * cache, which shares the KV cache's page indexing; "Sparse Attention for
+ * Long-Context LLMs: Evolution and Practical Deployment", section 7.3: cache
+ * writes must stay consistent with the index, so every KV write here also
+ * refreshes the block representation. The representation is the mean of the
+ * block's keys over the tokens present, in fp32.
+ *
+ *   k_new, v_new      : device [N_new][num_kv_heads][head_dim], kv->dtype. The
+ *                       rows of sequence b are cu_new[b] .. cu_new[b+1]-1.
+ *   cu_new            : device [batch+1] int32, non-decreasing, cu_new[0] = 0.
+ *   max_new_per_seq   : host bound on cu_new[b+1]-cu_new[b] (sizes the grid).
+ *
+ * kv->seq_lens must already count the new tokens: sequence b's new rows go to
+ * positions seq_lens[b]-n_b .. seq_lens[b]-1. Writes those rows into the pages
+ * named by page_table and recomputes, for each touched block j,
+ *   centroids[page(b, j)][g][:] = (sum of the keys present in block j) / count
+ * with a fixed summation order, so appending token by token gives the same
+ * bits as pooling the full block at once. Untouched blocks are not read.
+ */
+msa_status_t msa_build_block_cache(const msa_paged_kv_t* kv, const void* k_new, const void* v_new,
+                                   const int32_t* cu_new, int32_t max_new_per_seq,
+                                   msa_stream_t stream);
+
+/*
+ * msa_select_topk - exp-free per-group top-k block selection.
+ *
+ * Follows "MiniMax Sparse Attention", method paragraph (a light index branch
+ * scores KV blocks and independently keeps a top-k subset for each GQA group)
+ * and results paragraph (exp-free top-k). For query row r at position t and KV
+ * group g, with qbar = sum of the group's G query heads (fp32):
+ *   score_j = qbar . centroid_j          for complete past blocks j < t / B;
+ *   S(r, g) = {t / B} plus the min(k-1, t/B) best j under
+ *             (score descending, block index ascending).
+ *
+ *   q                 : device [num_rows][num_q_heads][head_dim], kv->dtype.
+ *   cu_q              : device [batch+1] int32 or NULL. With cu_q, the rows of
+ *                       sequence b are cu_q[b] .. cu_q[b+1]-1 and sit at the
+ *                       LAST n_b positions: seq_lens[b]-n_b .. seq_lens[b]-1.
+ *                       NULL means decode: num_rows == batch, row b at
+ *                       position seq_lens[b]-1.
+ *   max_rows_per_seq  : host bound on n_b (sizes the grid; 1 for decode).
+ *   block_idx         : device out [num_rows][num_kv_heads][top_k] int32, the
+ *                       selected logical blocks in ascending order, -1 padded.
+ *   block_score       : device out, same shape, fp32, or NULL: the score of
+ *                       each selected past block, +INF for the own block,
+ *                       -INF for padding.
+ *   workspace         : device scratch of msa_workspace_size(MSA_OP_SELECT,..)
+ *                       bytes (may be NULL when that size is 0).
+ */
+msa_status_t msa_select_topk(const msa_paged_kv_t* kv, const void* q, const int32_t* cu_q,
+                             int32_t num_rows, int32_t max_rows_per_seq, int32_t top_k,
+                             int32_t* block_idx, float* block_score, void* workspace,
+                             size_t workspace_bytes, msa_stream_t stream);
+
+/*
+ * msa_sparse_attn_prefill - exact attention of many query rows over their
+ * selected blocks.
+ *
+ * Follows "MiniMax Sparse Attention", method paragraph (exact blockwise sparse
+ * attention over the selected blocks only) and "Sparse Attention + Linear
+ * Backbones", section 5.5 (softmax(q k_sel^T / sqrt(d)) v_sel). For row r at
+ * position t and query head h in group g:
+ *   U    = tokens u of the blocks in block_idx[r][g] with u <= t,
+ *   out  = sum_{u in U} softmax_u(scale * q.k_u) v_u     (kv->dtype, RNE),
+ *   lse  = log sum_{u in U} exp(scale * q.k_u)           (fp32, may be NULL).
+ *
+ *   q, cu_q, num_rows, max_rows_per_seq : as for msa_select_topk (cu_q must
+ *                       not be NULL here).
+ *   block_idx         : device [num_rows][num_kv_heads][top_k] int32, as
+ *                       produced by msa_select_topk (ascending, -1 padded,
+ *                       every entry <= t / B).
+ *   out               : device [num_rows][num_q_heads][head_dim], kv->dtype.
+ *   lse               : device [num_rows][num_q_heads] fp32, or NULL.
+ *   workspace         : device scratch, msa_workspace_size(MSA_OP_PREFILL, ..).
+ */
+msa_status_t msa_sparse_attn_prefill(const msa_paged_kv_t* kv, const void* q, const int32_t* cu_q,
+                                     int32_t num_rows, int32_t max_rows_per_seq,
+                                     const int32_t* block_idx, int32_t top_k, float softmax_scale,
+                                     void* out, float* lse, void* workspace,
+                                     size_t workspace_bytes, msa_stream_t stream);
+
+/*
+ * msa_sparse_attn_decode - the same attention for one new query per sequence
+ * (position seq_lens[b]-1, its own token already appended), computed as
+ * split-k partials over the selected blocks and merged by log-sum-exp.
+ *
+ * Follows "Art of Focus: Ling 2.0 ...", "Summarizing the Breakthrough" (during
+ * decode only the top-k relevant blocks are fetched) and the attention rule
+ * above.
+ *
+ *   q                 : device [batch][num_q_heads][head_dim], kv->dtype.
+ *   block_idx         : device [batch][num_kv_heads][top_k] int32.
+ *   out, lse          : device [batch][num_q_heads][head_dim] / [batch][num_q_heads].
+ *   workspace         : device scratch, msa_workspace_size(MSA_OP_DECODE, ..).
+ */
+msa_status_t msa_sparse_attn_decode(const msa_paged_kv_t* kv, const void* q,
+                                    const int32_t* block_idx, int32_t top_k, float softmax_scale,
+                                    void* out, float* lse, void* workspace, size_t workspace_bytes,
+                                    msa_stream_t stream);
+
+/* Scratch bytes that `op` needs for these sizes (num_rows / max_rows_per_seq
+ * as passed to the op; batch and 1 for decode). 0 means no scratch. */
+size_t msa_workspace_size(msa_op_t op, const msa_paged_kv_t* kv, int32_t num_rows,
+                          int32_t max_rows_per_seq, int32_t top_k);
+
+/* Static, NUL-terminated description of a status code. */
+const char* msa_status_string(msa_status_t status);
+
+/* Library ABI version (major * 1000 + minor). */
+int32_t msa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MSA_H_ */

@@ -1,0 +1,311 @@
+"""GPU-vs-oracle parity on seeded inputs, through the C ABI (Python binding).
+
+Sizes here are small enough for the fp64 oracle to finish in seconds while
+spanning several query tiles, several blocks and ragged tails. Every input is
+drawn by the `workloads` generator on the GPU and independently regenerated on
+the CPU for the oracle (the generator is bit-identical across devices, which
+test_generator_bits_match checks).
+"""
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_gqa_mean_b200 as msa
+import oracle
+import workloads
+from msa_harness import (append, check_index_invariants, check_selection, compare, fill_context,
+                         new_cache, oracle_rows, read_pages)
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def test_library_loads_on_gpu():
+    assert torch.cuda.is_available()
+    assert msa.load_library().msa_version() >= 1000
+
+
+def test_generator_bits_match():
+    w = workloads.prefill_bf16()
+    for (u0, u1) in [(0, 300), (12345, 12400)]:
+        a = workloads.keys(w, 0, u0, u1, DEV).cpu()
+        b = workloads.keys(w, 0, u0, u1, "cpu")
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+        qa = workloads.queries_prefill(w, 0, u0, u1, DEV).cpu()
+        qb = workloads.queries_prefill(w, 0, u0, u1, "cpu")
+        assert torch.equal(qa.view(torch.int16), qb.view(torch.int16))
+    wt = workloads.tiny_f32()
+    assert torch.equal(workloads.keys(wt, 0, 0, 1024, DEV).cpu(), workloads.keys(wt, 0, 0, 1024))
+
+
+# ---------------------------------------------------------------------------
+# block cache
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_append_pool_matches_oracle_and_rebuild(dtype):
+    d, B = (128, 128) if dtype == "bf16" else (64, 64)
+    w = workloads.paged_decode_bf16(batch=3, ctx=(1000, 257, 3000), block=B, d=d, dtype=dtype,
+                                    hq=8, hkv=2, steps=0)
+    p = workloads.paging(w)
+    # one-shot build
+    c1 = new_cache(w, p)
+    append(c1, w, [0] * 3, list(w.ctx))
+    # ragged multi-call build: 1 token, then chunks, then singles
+    c2 = new_cache(w, p)
+    lens = [0, 0, 0]
+    for target in ([1, 1, 1], [130, 64, 700], [131, 200, 2999], list(w.ctx)):
+        append(c2, w, lens, target)
+        lens = target
+    torch.cuda.synchronize()
+    assert c1.device_status() == 0 and c2.device_status() == 0
+    assert torch.equal(c1.centroids, c2.centroids)  # same bits, whatever the append pattern
+    for b in range(3):
+        L = w.ctx[b]
+        K = workloads.keys(w, b, 0, L)
+        assert torch.equal(read_pages(c1, b, L, "k").view(torch.uint8), K.view(torch.uint8))
+        assert torch.equal(read_pages(c1, b, L, "v").view(torch.uint8),
+                           workloads.values(w, b, 0, L).view(torch.uint8))
+        C = oracle.centroids(K, B)
+        ids = p.table[b, :C.shape[0]].long()
+        got = c1.centroids.cpu()[ids].double().numpy()
+        # fp32 relative 1e-6, relative to the block's mean key magnitude (the
+        # scale of the rounding error of a sum of fp32 terms)
+        Kd = K.double().numpy()
+        nb = C.shape[0]
+        pad = np.zeros((nb * B - L,) + Kd.shape[1:])
+        scale = np.abs(np.concatenate([Kd, pad])).reshape(nb, B, w.hkv, d).sum(1)
+        scale /= np.minimum(B, L - np.arange(nb) * B)[:, None, None]
+        assert np.all(np.abs(got - C) <= 1e-6 * np.maximum(np.abs(C), scale.mean(-1, keepdims=True)))
+
+
+# ---------------------------------------------------------------------------
+# prefill: selection + attention
+# ---------------------------------------------------------------------------
+PREFILL_CASES = [
+    # (name, overrides)
+    ("g8_b128", dict(ctx=(1200,), top_k=4)),
+    ("g8_b128_k16", dict(ctx=(2200,), top_k=16)),
+    ("g16_b128", dict(ctx=(900,), hq=64, hkv=4, top_k=3)),
+    ("g8_b64", dict(ctx=(700,), block=64, top_k=5)),
+    ("g4_simt", dict(ctx=(500,), hq=16, hkv=4, top_k=3)),
+]
+
+
+def _run_prefill(w, cache, device=DEV):
+    T = w.ctx[0]
+    append(cache, w, [0], [T])
+    q = workloads.queries_prefill(w, 0, 0, T, device)
+    cu = msa.cu_seqlens([T], device)
+    idx, sc = msa.select_topk(cache, q, w.top_k, cu_q=cu, max_rows_per_seq=T, want_scores=True)
+    out, lse = msa.sparse_attn_prefill(cache, q, idx, cu_q=cu, max_rows_per_seq=T)
+    torch.cuda.synchronize()
+    return q, cu, idx, sc, out, lse
+
+
+@pytest.mark.parametrize("name,over", PREFILL_CASES, ids=[c[0] for c in PREFILL_CASES])
+def test_prefill_end_to_end(name, over):
+    w = workloads.prefill_bf16(**over)
+    p = workloads.paging(w)
+    cache = new_cache(w, p)
+    q, cu, idx, sc, out, lse = _run_prefill(w, cache)
+    assert cache.device_status() == 0
+    T = w.ctx[0]
+    pos = np.arange(T)
+    orc = oracle_rows(w, 0, T, pos, q.cpu())
+    stats = check_selection(idx.cpu().numpy(), orc, pos, w.top_k, w.block)
+    assert stats["protected_frac"] > 0.3
+    # attention checked on the oracle's own indices (removes tie ambiguity)
+    oi = torch.from_numpy(orc["idx"]).to(DEV)
+    out2, lse2 = msa.sparse_attn_prefill(cache, q, oi, cu_q=cu, max_rows_per_seq=T)
+    torch.cuda.synchronize()
+    compare(out2, orc["out"], w.dtype)
+    assert np.abs(lse2.cpu().double().numpy() - orc["lse"]).max() < 2e-3
+    # where the selections agree the end-to-end output matches too
+    same = (idx.cpu().numpy() == orc["idx"]).all(-1)             # [T, Hkv]
+    rows_ok = same.all(-1)
+    assert rows_ok.mean() > 0.5
+    compare(out[torch.from_numpy(rows_ok).to(DEV)], orc["out"][rows_ok], w.dtype)
+
+
+def test_tiny_f32_prefill_and_decode():
+    """The tiny fp32 workload: full prefill of 1024 rows, then decode of the last
+    query after 1023 cached tokens; decode must equal prefill row 1023."""
+    w = workloads.tiny_f32()
+    p = workloads.paging(w)
+    cache = new_cache(w, p)
+    q, cu, idx, sc, out, lse = _run_prefill(w, cache)
+    T = w.ctx[0]
+    pos = np.arange(T)
+    orc = oracle_rows(w, 0, T, pos, q.cpu())
+    check_selection(idx.cpu().numpy(), orc, pos, w.top_k, w.block)
+    oi = torch.from_numpy(orc["idx"]).to(DEV)
+    out2, lse2 = msa.sparse_attn_prefill(cache, q, oi, cu_q=cu, max_rows_per_seq=T)
+    torch.cuda.synchronize()
+    compare(out2, orc["out"], "f32")
+    assert np.abs(lse2.cpu().double().numpy() - orc["lse"]).max() < 1e-5
+    # decode: cache of 1023 tokens, append token 1023, attend
+    c2 = new_cache(w, p)
+    append(c2, w, [0], [T - 1])
+    append(c2, w, [T - 1], [T])
+    qd = q[T - 1:].contiguous()
+    di, _ = msa.select_topk(c2, qd, w.top_k)
+    do, dl = msa.sparse_attn_decode(c2, qd, di)
+    torch.cuda.synchronize()
+    assert torch.equal(di, idx[T - 1:])
+    compare(do, orc["out"][T - 1:], "f32")
+    assert torch.allclose(do, out[T - 1:], atol=1e-6, rtol=0)
+
+
+def test_prefill_page_permutation_invariance():
+    w = workloads.prefill_bf16(ctx=(1100,), top_k=5)
+    p1 = workloads.paging(w)
+    p2 = workloads.paging(w, spare_pages=7)   # different pool size -> different permutation
+    assert not torch.equal(p1.table, p2.table[:, :p1.table.shape[1]])
+    r1 = _run_prefill(w, new_cache(w, p1))
+    r2 = _run_prefill(w, new_cache(w, p2))
+    assert torch.equal(r1[2], r2[2])
+    assert torch.equal(r1[4].view(torch.int16), r2[4].view(torch.int16))
+
+
+def test_chunked_prefill_matches_full():
+    """Rows appended in two chunks (q_pos0 > 0 through cu_q + seq_lens) equal the
+    same rows of a one-shot prefill."""
+    w = workloads.prefill_bf16(ctx=(1500,), top_k=6)
+    p = workloads.paging(w)
+    full = _run_prefill(w, new_cache(w, p))
+    cache = new_cache(w, p)
+    T, T0 = 1500, 1000
+    append(cache, w, [0], [T0])
+    append(cache, w, [T0], [T])
+    q = workloads.queries_prefill(w, 0, T0, T, DEV)
+    cu = msa.cu_seqlens([T - T0], DEV)
+    idx, _ = msa.select_topk(cache, q, w.top_k, cu_q=cu, max_rows_per_seq=T - T0)
+    out, _ = msa.sparse_attn_prefill(cache, q, idx, cu_q=cu, max_rows_per_seq=T - T0)
+    torch.cuda.synchronize()
+    assert torch.equal(idx, full[2][T0:])
+    compare(out, full[4][T0:].float().cpu().double().numpy(), "bf16")
+
+
+# ---------------------------------------------------------------------------
+# decode
+# ---------------------------------------------------------------------------
+DECODE_CASES = [
+    ("paged_g4", lambda: workloads.paged_decode_bf16(batch=4, ctx=(3000, 4095, 4096, 5000))),
+    ("long_g8_b128", lambda: workloads.decode_1m_bf16(ctx=(40000,), steps=3)),
+    ("varlen_g16", lambda: workloads.varlen_decode_bf16(batch=5, len_range=(1000, 20000))),
+]
+
+
+@pytest.mark.parametrize("name,make", DECODE_CASES, ids=[c[0] for c in DECODE_CASES])
+def test_decode_end_to_end(name, make):
+    w = make()
+    p = workloads.paging(w)
+    cache = new_cache(w, p)
+    lens = fill_context(cache, w)
+    hit = [0, 0]   # planted blocks selected / planted blocks
+    for step in range(w.steps):
+        after = [w.ctx[b] + step + 1 for b in range(w.batch)]
+        append(cache, w, lens, after)
+        lens = after
+        q = workloads.queries_decode(w, step, DEV)
+        idx, _ = msa.select_topk(cache, q, w.top_k)
+        out, lse = msa.sparse_attn_decode(cache, q, idx)
+        torch.cuda.synchronize()
+        assert cache.device_status() == 0
+        oidx, refs = [], []
+        for b in range(w.batch):
+            L = lens[b]
+            pos = np.array([L - 1])
+            K, V = workloads.keys(w, b, 0, L), workloads.values(w, b, 0, L)
+            orc = oracle.forward(q[b:b + 1].cpu(), K, V, pos, w.block, w.top_k, w.softmax_scale)
+            check_selection(idx[b:b + 1].cpu().numpy(), orc, pos, w.top_k, w.block)
+            for g, blocks in enumerate(workloads.planted_blocks(w)[b]):
+                hit[0] += len(set(blocks) & set(idx[b, g].tolist()))
+                hit[1] += len(blocks)
+            if np.array_equal(orc["idx"], idx[b:b + 1].cpu().numpy()):
+                compare(out[b:b + 1], orc["out"], w.dtype)
+                assert np.abs(lse[b].cpu().double().numpy() - orc["lse"][0]).max() < 2e-3
+            oidx.append(orc["idx"])
+            refs.append(orc["out"])
+        # attention on the oracle's indices, all sequences at once
+        o2, _ = msa.sparse_attn_decode(cache, q, torch.from_numpy(np.concatenate(oidx)).to(DEV))
+        torch.cuda.synchronize()
+        compare(o2, np.concatenate(refs), w.dtype)
+    # the planted "needle" blocks are found far more often than chance
+    assert hit[1] == 0 or hit[0] >= 0.75 * hit[1], hit
+
+
+def test_decode_equals_prefill_rows():
+    """Selecting and attending the last rows one at a time through the decode
+    entry points gives the prefill selection and (within bf16 tolerance) output."""
+    w = workloads.prefill_bf16(ctx=(1300,), top_k=5, hq=16, hkv=2)
+    p = workloads.paging(w)
+    full = _run_prefill(w, new_cache(w, p))
+    cache = new_cache(w, p)
+    T = 1300
+    append(cache, w, [0], [T - 3])
+    for t in range(T - 3, T):
+        append(cache, w, [t], [t + 1])
+        q = full[0][t:t + 1].contiguous()
+        di, _ = msa.select_topk(cache, q, w.top_k)
+        do, _ = msa.sparse_attn_decode(cache, q, di)
+        torch.cuda.synchronize()
+        assert torch.equal(di, full[2][t:t + 1])
+        compare(do, full[4][t:t + 1].float().cpu().double().numpy(), "bf16")
+
+
+# ---------------------------------------------------------------------------
+# error paths (no fault, no trap: host status codes and the device status word)
+# ---------------------------------------------------------------------------
+def test_host_argument_errors():
+    w = workloads.prefill_bf16(ctx=(256,), top_k=2)
+    p = workloads.paging(w)
+    cache = new_cache(w, p)
+    append(cache, w, [0], [256])
+    q = workloads.queries_prefill(w, 0, 0, 256, DEV)
+    cu = msa.cu_seqlens([256], DEV)
+    with pytest.raises(msa.MsaError) as e:
+        msa.select_topk(cache, q, 0, cu_q=cu, max_rows_per_seq=256)
+    assert e.value.status == msa.MSA_ERR_UNSUPPORTED
+    with pytest.raises(msa.MsaError) as e:
+        msa.select_topk(cache, q, 300, cu_q=cu, max_rows_per_seq=256)
+    assert e.value.status == msa.MSA_ERR_UNSUPPORTED
+    idx, _ = msa.select_topk(cache, q, 2, cu_q=cu, max_rows_per_seq=256)
+    small = torch.empty(16, dtype=torch.uint8, device=DEV)
+    with pytest.raises(msa.MsaError) as e:
+        msa.sparse_attn_prefill(cache, q, idx, cu_q=cu, max_rows_per_seq=256, workspace=small)
+    assert e.value.status == msa.MSA_ERR_WORKSPACE
+    bad = msa.PagedKVCache(cache.k_pages, cache.v_pages, cache.centroids, cache.page_table,
+                           cache.seq_lens, cache.status_word, num_q_heads=33)
+    with pytest.raises(msa.MsaError) as e:
+        msa.select_topk(bad, q, 2, cu_q=cu, max_rows_per_seq=256)
+    assert e.value.status == msa.MSA_ERR_INVALID_ARG
+    torch.cuda.synchronize()
+    assert cache.device_status() == 0
+
+
+def test_device_status_on_bad_page_and_length():
+    w = workloads.paged_decode_bf16(batch=2, ctx=(500, 700))
+    p = workloads.paging(w)
+    cache = new_cache(w, p)
+    fill_context(cache, w)
+    append(cache, w, list(w.ctx), [w.ctx[0] + 1, w.ctx[1] + 1])
+    q = workloads.queries_decode(w, 0, DEV)
+    cache.page_table[1, 3] = p.num_pages + 5          # corrupt one page id (host-side injection)
+    idx, _ = msa.select_topk(cache, q, w.top_k)
+    msa.sparse_attn_decode(cache, q, idx)
+    torch.cuda.synchronize()
+    assert cache.device_status() & msa.MSA_DEV_BAD_PAGE
+    cache.clear_status()
+    cache.page_table.copy_(p.table.to(DEV))
+    cache.seq_lens[0] = p.max_blocks * w.block + 1    # beyond capacity
+    idx, _ = msa.select_topk(cache, q, w.top_k)
+    torch.cuda.synchronize()
+    assert cache.device_status() & msa.MSA_DEV_BAD_LENGTH
+    # the context still works afterwards
+    cache.clear_status()
+    cache.seq_lens.copy_(torch.tensor([w.ctx[0] + 1, w.ctx[1] + 1], dtype=torch.int32))
+    idx, _ = msa.select_topk(cache, q, w.top_k)
+    msa.sparse_attn_decode(cache, q, idx)
+    torch.cuda.synchronize()
+    assert cache.device_status() == 0
