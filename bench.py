@@ -433,11 +433,15 @@ def main():
     ap.add_argument("--no-decode", action="store_true", help="skip the paged-decode block")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--oracle-rows", type=int, default=256)
+    ap.add_argument("--seq-len", type=int, default=0,
+                    help="override the prefill length (profiling of a smaller case)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     world, rank, local = dist_setup()
     w = workloads.ALL[args.workload]()
+    if args.seq_len and w.kind == "prefill":
+        w = workloads.ALL[args.workload](ctx=(args.seq_len,))
     pk = peaks()
 
     if args.impl == "reference":
