@@ -33,7 +33,8 @@ MSA_OP_SELECT, MSA_OP_PREFILL, MSA_OP_DECODE = 0, 1, 2
 MSA_DEV_BAD_PAGE, MSA_DEV_BAD_LENGTH, MSA_DEV_BAD_INDEX, MSA_DEV_TIMEOUT = 1, 2, 4, 8
 
 EXPORTS = ("msa_build_block_cache", "msa_select_topk", "msa_sparse_attn_prefill",
-           "msa_sparse_attn_decode", "msa_workspace_size", "msa_status_string", "msa_version")
+           "msa_sparse_attn_decode", "msa_sparse_attn_decode_noalloc", "msa_workspace_size",
+           "msa_status_string", "msa_version")
 
 
 class MsaError(RuntimeError):
@@ -80,13 +81,14 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.msa_sparse_attn_prefill.argtypes = [KV, P, P, I32, I32, P, I32, ctypes.c_float, P, P, P,
                                             SZ, P]
     lib.msa_sparse_attn_decode.argtypes = [KV, P, P, I32, ctypes.c_float, P, P, P, SZ, P]
+    lib.msa_sparse_attn_decode_noalloc.argtypes = [KV, P, P, I32, ctypes.c_float, P, P, P]
     lib.msa_workspace_size.argtypes = [ctypes.c_int, KV, I32, I32, I32]
     lib.msa_workspace_size.restype = SZ
     lib.msa_status_string.argtypes = [ctypes.c_int]
     lib.msa_status_string.restype = ctypes.c_char_p
     lib.msa_version.restype = I32
     for name in ("msa_build_block_cache", "msa_select_topk", "msa_sparse_attn_prefill",
-                 "msa_sparse_attn_decode"):
+                 "msa_sparse_attn_decode", "msa_sparse_attn_decode_noalloc"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -273,6 +275,25 @@ def sparse_attn_decode(cache: PagedKVCache, q: torch.Tensor, block_idx: torch.Te
     _check(lib.msa_sparse_attn_decode(ctypes.byref(kv), _ptr(q), _ptr(block_idx), top_k, scale,
                                       _ptr(out), _ptr(lse), _ptr(ws), ws_bytes, _stream(stream)),
            "msa_sparse_attn_decode")
+    return out, lse
+
+
+def sparse_attn_decode_noalloc(cache: PagedKVCache, q: torch.Tensor, block_idx: torch.Tensor,
+                               out: torch.Tensor, lse: Optional[torch.Tensor] = None,
+                               softmax_scale: Optional[float] = None, stream=None):
+    """sparse_attn_decode for callers that cannot allocate device memory: the
+    caller passes the outputs, and the split-k scratch is the library's own
+    8 MiB device array (shared by every call on the device, so calls must not
+    overlap on the GPU). Raises MsaError(MSA_ERR_WORKSPACE) when the problem
+    needs more scratch than that."""
+    lib = load_library()
+    _require_cuda(q, block_idx, out, lse)
+    top_k = block_idx.shape[-1]
+    scale = 1.0 / math.sqrt(cache.head_dim) if softmax_scale is None else softmax_scale
+    kv = cache.struct()
+    _check(lib.msa_sparse_attn_decode_noalloc(ctypes.byref(kv), _ptr(q), _ptr(block_idx), top_k,
+                                              scale, _ptr(out), _ptr(lse), _stream(stream)),
+           "msa_sparse_attn_decode_noalloc")
     return out, lse
 
 

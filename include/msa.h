@@ -207,6 +207,32 @@ msa_status_t msa_sparse_attn_decode(const msa_paged_kv_t* kv, const void* q,
                                     void* out, float* lse, void* workspace, size_t workspace_bytes,
                                     msa_stream_t stream);
 
+/*
+ * msa_sparse_attn_decode_noalloc - msa_sparse_attn_decode for callers that
+ * cannot allocate device memory at the call: a plugin run by a host framework
+ * that owns the device memory pool and offers no scratch allocator, or a
+ * latency-bound loop that must not call the allocator. The pages describe no
+ * such call; it exists for those callers only.
+ *
+ * Same arguments and results as msa_sparse_attn_decode minus the workspace:
+ * the split-k partials go to one 8 MiB device array inside libmsa.so, which
+ * every GPU that loads the library keeps until the process exits.
+ *  - Returns MSA_ERR_WORKSPACE, launching nothing, when the problem needs more
+ *    than 8 MiB, i.e. when msa_workspace_size(MSA_OP_DECODE, kv, batch, 1,
+ *    top_k) > 8 MiB (about batch * num_q_heads * splits * 516 bytes).
+ *  - All calls on a device share the array: calls whose kernels may overlap
+ *    on the GPU (unordered streams) race; calls on one stream do not. Nothing
+ *    in the array needs to start at zero.
+ *  - The first call on each device resolves the array's device address
+ *    (cudaGetSymbolAddress, with that device current); make it before any
+ *    stream capture.
+ *  - Allocates nothing: no cudaMalloc, no cudaFree, no allocating library call.
+ */
+msa_status_t msa_sparse_attn_decode_noalloc(const msa_paged_kv_t* kv, const void* q,
+                                            const int32_t* block_idx, int32_t top_k,
+                                            float softmax_scale, void* out, float* lse,
+                                            msa_stream_t stream);
+
 /* Scratch bytes that `op` needs for these sizes (num_rows / max_rows_per_seq
  * as passed to the op; batch and 1 for decode). 0 means no scratch. */
 size_t msa_workspace_size(msa_op_t op, const msa_paged_kv_t* kv, int32_t num_rows,
