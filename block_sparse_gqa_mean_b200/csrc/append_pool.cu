@@ -9,9 +9,9 @@
 // re-pools the centroid of the block it lands in, in the same kernel.
 //
 // One CTA per (sequence, touched block, KV head). It copies the new rows of
-// that block into the page (16-byte vector copies), then every thread owns
-// one coordinate and sums the keys present in the block in token order, in
-// fp32, and divides by the count. The order does not depend on how the tokens
+// that block into the page (16-byte vector copies), stages the block's keys
+// in shared memory, then every thread owns one coordinate and sums the keys
+// present in the block in token order, in fp32, and divides by the count. The order does not depend on how the tokens
 // arrived, so token-by-token appends and a one-shot build give equal bits.
 #include "common.cuh"
 
@@ -60,12 +60,18 @@ __global__ void __launch_bounds__(128) append_pool_kernel(
   }
   __syncthreads();
 
-  // 2) re-pool the block: mean over every token present, fixed token order
+  // 2) re-pool the block: mean over every token present, fixed token order.
+  //    The block's keys are staged in shared memory with 16-byte loads first.
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  T* tile = reinterpret_cast<T*>(smem_raw);  // [n][D]
   const int n = u_hi - j * B;
+  for (int c = threadIdx.x; c < n * CPR; c += blockDim.x)
+    reinterpret_cast<uint4*>(tile)[c] =
+        reinterpret_cast<const uint4*>(k_pages + page_off)[c];
+  __syncthreads();
   for (int i = threadIdx.x; i < D; i += blockDim.x) {
-    const T* col = k_pages + page_off + i;
     float s = 0.f;
-    for (int u = 0; u < n; ++u) s = __fadd_rn(s, to_f32(col[(size_t)u * D]));
+    for (int u = 0; u < n; ++u) s = __fadd_rn(s, to_f32(tile[u * D + i]));
     centroids[((size_t)page * hkv + g) * D + i] = __fdiv_rn(s, (float)n);
   }
 }
@@ -75,7 +81,11 @@ static cudaError_t launch_append(const msa_paged_kv_t* kv, const void* k_new, co
                                  const int32_t* cu_new, int max_new, cudaStream_t st) {
   const int B = kv->block_size;
   dim3 grid((max_new + B - 1) / B + 1, kv->batch, kv->num_kv_heads);
-  append_pool_kernel<T, D><<<grid, 128, 0, st>>>(
+  const size_t smem = (size_t)B * D * sizeof(T);
+  cudaError_t e = cudaFuncSetAttribute(append_pool_kernel<T, D>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  append_pool_kernel<T, D><<<grid, 128, smem, st>>>(
       (const T*)k_new, (const T*)v_new, cu_new, (T*)kv->k_pages, (T*)kv->v_pages, kv->centroids,
       kv->page_table, kv->seq_lens, kv->status_word, kv->num_kv_heads, B, kv->num_pages,
       kv->max_blocks_per_seq);

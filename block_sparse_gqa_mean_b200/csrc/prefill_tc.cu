@@ -9,21 +9,25 @@
 // Work unit: a query tile of TM = 128 / G consecutive tokens of one sequence
 // and one KV group, i.e. 128 query rows (token-major, the group's G heads per
 // token). The tile's tokens select their blocks independently, so the tile
-// walks the UNION of their selections (built by prefill_plan_kernel, ascending,
-// each entry carrying a bit per token that selected it). Per union block the
-// CTA computes S = Q K^T for all 128 rows on the tensor cores and the softmax
-// gives zero weight to rows whose token did not select the block.
+// walks the UNION of their selections (built by prefill_plan_kernel,
+// ascending, each entry carrying one bit per token). Per union block the CTA
+// computes S = Q K^T for all 128 rows on the tensor cores and the softmax
+// gives zero weight to the rows of tokens that did not select the block.
 //
 // CTA layout (192 threads): warp 0 issues TMA loads of K and V tiles (two
-// 64-column boxes each, 128-byte swizzle, no multicast) into a 3-stage ring;
-// warp 1 owns the TMEM allocation and issues tcgen05.mma from one thread;
-// warps 2..5 are the softmax warps, one TMEM lane (query row) per thread.
-// TMEM columns: Q (bf16, A operand) | P (bf16, A operand) | S0 | S1 | O (fp32).
-//   S = Q K^T : M=128, N=B, K=128, A = Q from TMEM, B = K tile (K-major SW128)
-//   O += P V  : M=128, N=128, K=B, A = P from TMEM, B = V tile (MN-major SW128)
-// S is double-buffered so the tensor cores compute S for block e+1 while the
-// softmax warps exponentiate block e. The online softmax rescales O in TMEM
-// only when a row's running max grows.
+// 64-column boxes each, 128-byte swizzle, no multicast) into a ring of
+// stages; warp 1 owns the TMEM allocation and issues tcgen05.mma from one
+// thread; warps 2..5 are the softmax warps, one TMEM lane (query row) per
+// thread.
+//   TMEM columns : Q (bf16 pairs, 64) | P0 | P1 (bf16 pairs, 64 each) |
+//                  S (fp32, 128) | O (fp32, 128)
+//   S = Q K^T    : M=128, N=B, K=128, A = Q (TMEM), B = K tile (K-major SW128)
+//   O += P V     : M=128, N=128, K=B, A = P (TMEM), B = V tile (MN-major SW128)
+// The softmax reads S into registers at once and releases it, so the tensor
+// cores compute S for block e+1 while the exponentials of block e run; P is
+// double-buffered and the softmax reference max moves lazily (only when a
+// row's max grows by more than 2^8), so writing P never waits for the P V in
+// flight and O is rescaled in TMEM only rarely.
 #include "tma.cuh"
 
 namespace msa {
@@ -33,11 +37,6 @@ namespace {
 constexpr int kD = 128;
 constexpr float kLog2e = 1.4426950408889634f;
 
-// TMEM column map (512 columns allocated)
-constexpr uint32_t kColQ = 0;     // 64 columns: 128 bf16 per row
-constexpr uint32_t kColP = 64;    // 64 columns: up to 128 bf16 per row
-constexpr uint32_t kColS = 128;   // two 128-column fp32 buffers
-constexpr uint32_t kColO = 384;   // 128 columns fp32
 
 // ---- tcgen05 wrappers ------------------------------------------------------
 __device__ __forceinline__ void tc_fence_before() {
@@ -126,31 +125,34 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 }  // namespace
 
 // ---------------------------------------------------------------------------
-// Planning: union of each tile's selections, ascending, with token bitmasks.
+// Planning: for each unit of query tiles (tiles_per_unit * TM consecutive
+// tokens), the union of the tokens' selections, ascending, each block with a
+// 32-bit mask: bit (tile * 16 + token-in-tile) is set when that token selected
+// the block.
 // ---------------------------------------------------------------------------
 constexpr int kPlanWindow = 4096;
 
 __global__ void __launch_bounds__(128) prefill_plan_kernel(
     const int32_t* __restrict__ cu_q, const int32_t* __restrict__ seq_lens,
     const int32_t* __restrict__ block_idx, uint32_t* status, int hkv, int B, int max_blocks,
-    int top_k, int TM, int tiles_per_seq, int ecap, int2* __restrict__ entries,
-    int* __restrict__ counts) {
+    int top_k, int TM, int tiles_per_unit, int units_per_seq, int ecap,
+    int2* __restrict__ entries, int* __restrict__ counts) {
   __shared__ uint32_t bm[kPlanWindow];
   __shared__ int warp_tot[4];
   __shared__ int s_base;
-  const int tile = blockIdx.x;
+  const int tile = blockIdx.x;  // unit index
   const int g = tile % hkv;
-  const int tt = (tile / hkv) % tiles_per_seq;
-  const int b = tile / (hkv * tiles_per_seq);
+  const int tt = (tile / hkv) % units_per_seq;
+  const int b = tile / (hkv * units_per_seq);
   const int tid = threadIdx.x, lane = tid % 32, warp = tid / 32;
   const int row0 = cu_q[b];
   const int n_rows = cu_q[b + 1] - row0;
-  const int r_lo = tt * TM;
+  const int r_lo = tt * tiles_per_unit * TM;
   if (r_lo >= n_rows) {
     if (tid == 0) counts[tile] = 0;
     return;
   }
-  const int nr = min(TM, n_rows - r_lo);
+  const int nr = min(tiles_per_unit * TM, n_rows - r_lo);
   const int L = seq_lens[b];
   if (n_rows > L || L > max_blocks * B) {
     if (tid == 0) {
@@ -177,7 +179,7 @@ __global__ void __launch_bounds__(128) prefill_plan_kernel(
         report(status, MSA_DEV_BAD_INDEX);
         continue;
       }
-      if (j >= w0 && j < w0 + W) atomicOr(&bm[j - w0], 1u << i);
+      if (j >= w0 && j < w0 + W) atomicOr(&bm[j - w0], 1u << ((i / TM) * 16 + i % TM));
     }
     __syncthreads();
     // compaction: thread tid scans words [tid*per, (tid+1)*per)
@@ -206,39 +208,65 @@ __global__ void __launch_bounds__(128) prefill_plan_kernel(
 // ---------------------------------------------------------------------------
 // Attention
 // ---------------------------------------------------------------------------
+constexpr float kRescaleLog2 = 8.f;  // lazy rescale threshold (log2 units)
+
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  return ((uint64_t)__float_as_uint(hi) << 32) | __float_as_uint(lo);
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 template <int B, int G>
 __global__ void __launch_bounds__(192, 1) prefill_tc_kernel(
     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
     const bf16* __restrict__ q, const int32_t* __restrict__ cu_q,
     const int32_t* __restrict__ page_table, const int32_t* __restrict__ seq_lens, uint32_t* status,
-    int hq, int hkv, int num_pages, int max_blocks, int tiles_per_seq, int ecap,
+    int hq, int hkv, int num_pages, int max_blocks, int units_per_seq, int ecap,
     const int2* __restrict__ entries, const int* __restrict__ counts, float scale_log2,
     bf16* __restrict__ out, float* __restrict__ lse) {
-  constexpr int TM = 128 / G;            // tokens per tile
-  constexpr int NST = (B == 128) ? 3 : 4;
-  constexpr int TILE = B * kD * 2;       // bytes of a K (or V) tile
+  constexpr int TM = 128 / G;              // tokens per query tile (128 rows)
+  constexpr int NST = (B == 128) ? 3 : 4;  // K+V stages
+  constexpr int TILE = B * kD * 2;         // bytes of a K (or V) tile
   constexpr int STAGE = 2 * TILE;
   constexpr uint32_t IDESC_S = idesc_bf16(128, B, false);
   constexpr uint32_t IDESC_O = idesc_bf16(128, kD, true);
+  // TMEM columns
+  constexpr uint32_t COL_Q = 0;    // Q, 64 columns (bf16 pairs), A operand of S = Q K^T
+  constexpr uint32_t COL_P = 64;   // two P buffers of 64 columns (bf16 pairs)
+  constexpr uint32_t COL_S = 192;  // S, 128 columns (fp32)
+  constexpr uint32_t COL_O = 320;  // O, 128 columns (fp32)
 
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  unsigned char* smem = reinterpret_cast<unsigned char*>(
+  unsigned char* stages = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   __shared__ __align__(8) uint64_t kv_full[NST], kv_empty[NST];
-  __shared__ __align__(8) uint64_t s_full[2], s_free[2], p_full, o_done, q_ready, fin;
+  __shared__ __align__(8) uint64_t s_full, s_free, p_full[2], o_done[2], q_ready, fin;
   __shared__ uint32_t s_tmem;
   __shared__ volatile int s_abort;
 
-  const int tile = blockIdx.x;
-  const int g = tile % hkv;
-  const int tt = (tile / hkv) % tiles_per_seq;
-  const int b = tile / (hkv * tiles_per_seq);
-  const int n_e = counts[tile];
-  if (n_e == 0) return;  // empty tile (ragged batch) - uniform exit before any sync
-  const int2* ent = entries + (size_t)tile * ecap;
+  const int unit = blockIdx.x;
+  const int g = unit % hkv;
+  const int pu = (unit / hkv) % units_per_seq;
+  const int b = unit / (hkv * units_per_seq);
+  const int n_e = counts[unit];
+  if (n_e == 0) return;  // nothing to do (ragged batch) - uniform exit before any sync
+  const int2* ent = entries + (size_t)unit * ecap;
   const int row0 = cu_q[b];
   const int n_rows = cu_q[b + 1] - row0;
-  const int r_lo = tt * TM;
+  const int r_lo = pu * TM;
   const int nr = min(TM, n_rows - r_lo);
   const int L = seq_lens[b];
   const int t_first = L - n_rows + r_lo;
@@ -249,12 +277,12 @@ __global__ void __launch_bounds__(192, 1) prefill_tc_kernel(
       mbar_init(&kv_full[s], 1);
       mbar_init(&kv_empty[s], 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&s_full[s], 1);
-      mbar_init(&s_free[s], 128);
+    mbar_init(&s_full, 1);
+    mbar_init(&s_free, 128);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&p_full[x], 128);
+      mbar_init(&o_done[x], 1);
     }
-    mbar_init(&p_full, 128);
-    mbar_init(&o_done, 1);
     mbar_init(&q_ready, 128);
     mbar_init(&fin, 1);
     s_abort = 0;
@@ -286,10 +314,10 @@ __global__ void __launch_bounds__(192, 1) prefill_tc_kernel(
         int pg = page_table[(size_t)b * max_blocks + j];
         if (pg < 0 || pg >= num_pages) {
           report(status, MSA_DEV_BAD_PAGE);
-          pg = 0;  // keep the pipeline in step; the result of this tile is unspecified
+          pg = 0;  // keep the pipeline in step; the result of this unit is unspecified
         }
         const int y = (pg * hkv + g) * B;
-        unsigned char* kt = smem + st * STAGE;
+        unsigned char* kt = stages + st * STAGE;
         mbar_expect_tx(&kv_full[st], STAGE);
         tma_load_2d(kt, &tm_k, &kv_full[st], 0, y);
         tma_load_2d(kt + TILE / 2, &tm_k, &kv_full[st], 64, y);
@@ -302,41 +330,41 @@ __global__ void __launch_bounds__(192, 1) prefill_tc_kernel(
         if (!mbar_wait(&kv_full[e % NST], (e / NST) & 1)) report(status, MSA_DEV_TIMEOUT);
     }
   } else if (warp == 1) {
-    // ---------------- MMA issuer ----------------
+    // ---------------- MMA issuer (one thread) ----------------
     if (lane == 0) {
       bool ok = mbar_wait(&q_ready, 0);
       tc_fence_after();
+      // S_e = Q K_e^T, once block e is loaded and the softmax has read S_{e-1}
       auto issue_s = [&](int e) -> bool {
-        const int st = e % NST, sb = e & 1;
+        const int st = e % NST;
         if (!mbar_wait(&kv_full[st], (e / NST) & 1)) return false;
-        if (!mbar_wait(&s_free[sb], ((e >> 1) & 1) ^ 1)) return false;
+        if (e >= 1 && !mbar_wait(&s_free, (e - 1) & 1)) return false;
         tc_fence_after();
-        const uint32_t kt = smem_u32(smem + st * STAGE);
+        const uint32_t kt = smem_u32(stages + st * STAGE);
 #pragma unroll
         for (int ks = 0; ks < kD / 16; ++ks) {
-          const uint32_t addr = kt + (uint32_t)(ks >> 2) * (uint32_t)(TILE / 2) + (uint32_t)(ks & 3) * 32u;
-          tc_mma_ts(tmem + kColS + sb * 128, tmem + kColQ + ks * 8, sdesc_sw128(addr, 16, 1024),
+          const uint32_t boff = (uint32_t)(ks >> 2) * (uint32_t)(TILE / 2) + (uint32_t)(ks & 3) * 32u;
+          tc_mma_ts(tmem + COL_S, tmem + COL_Q + ks * 8, sdesc_sw128(kt + boff, 16, 1024),
                     IDESC_S, ks > 0);
         }
-        tc_commit(&s_full[sb]);
+        tc_commit(&s_full);
         return true;
       };
       if (ok) ok = issue_s(0);
       for (int e = 0; e < n_e && ok && !s_abort; ++e) {
-        if (e + 1 < n_e) ok = issue_s(e + 1);
-        if (!ok) break;
-        if (!mbar_wait(&p_full, e & 1)) { ok = false; break; }
+        if (e + 1 < n_e && !issue_s(e + 1)) { ok = false; break; }
+        const int pb = e & 1;
+        if (!mbar_wait(&p_full[pb], (e >> 1) & 1)) { ok = false; break; }
         tc_fence_after();
-        const int st = e % NST;
-        const uint32_t vt = smem_u32(smem + st * STAGE + TILE);
+        const uint32_t vt = smem_u32(stages + (e % NST) * STAGE + TILE);
 #pragma unroll
         for (int kk = 0; kk < B / 16; ++kk) {
-          tc_mma_ts(tmem + kColO, tmem + kColP + kk * 8,
+          tc_mma_ts(tmem + COL_O, tmem + COL_P + pb * 64 + kk * 8,
                     sdesc_sw128(vt + (uint32_t)kk * 2048u, (uint32_t)(TILE / 2), 1024), IDESC_O,
                     (e > 0 || kk > 0) ? 1u : 0u);
         }
-        tc_commit(&o_done);
-        tc_commit(&kv_empty[st]);
+        tc_commit(&o_done[pb]);
+        tc_commit(&kv_empty[e % NST]);
       }
       if (!ok) {
         report(status, MSA_DEV_TIMEOUT);
@@ -347,13 +375,13 @@ __global__ void __launch_bounds__(192, 1) prefill_tc_kernel(
       if (!mbar_wait(&fin, 0)) report(status, MSA_DEV_TIMEOUT);
     }
   } else {
-    // ---------------- softmax warps ----------------
+    // ---------------- softmax warps: a TMEM lane (query row) per thread ----------------
     const int quarter = warp & 3;
-    const int r = quarter * 32 + lane;           // query row of this thread == TMEM lane
+    const int r = quarter * 32 + lane;             // row within the tile == TMEM lane
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
-    const int ti = r / G, h = r % G;             // token within the tile, head within the group
+    const int ti = r / G, h = r % G;               // token within the tile, head in the group
     const bool row_ok = ti < nr;
-    const int t = t_first + ti;                   // position of this row's token
+    const int t = t_first + ti;                    // position of this row's token
     // Q row -> TMEM (bf16 pairs as 32-bit columns)
     {
       uint32_t qv[32];
@@ -363,108 +391,133 @@ __global__ void __launch_bounds__(192, 1) prefill_tc_kernel(
       for (int half = 0; half < 2; ++half) {
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
-          uint4 v = row_ok ? src[half * 8 + c] : make_uint4(0u, 0u, 0u, 0u);
+          const uint4 v = row_ok ? src[half * 8 + c] : make_uint4(0u, 0u, 0u, 0u);
           qv[4 * c + 0] = v.x;
           qv[4 * c + 1] = v.y;
           qv[4 * c + 2] = v.z;
           qv[4 * c + 3] = v.w;
         }
-        tc_st32(lane_base + kColQ + half * 32, qv);
+        tc_st32(lane_base + COL_Q + half * 32, qv);
       }
       tc_wait_st();
       tc_fence_before();
       mbar_arrive(&q_ready);
     }
-    float m = -INFINITY, l = 0.f;
+    // Online softmax with a lazily moved reference (log2 units): P = exp2(s*c - m_ref);
+    // m_ref moves, and O, l are rescaled, only when a row's max exceeds m_ref by
+    // more than kRescaleLog2, so the weights stay below 2^8 and writing P never
+    // has to wait for the P*V in flight. Rows whose token did not select the
+    // block use m = +inf, which turns every weight into an exact 0.
+    float m_ref = -INFINITY;
+    uint64_t l2 = f2_pack(0.f, 0.f);               // row sum, two fp32 lanes
+    const uint64_t sl2 = f2_pack(scale_log2, scale_log2);
     for (int e = 0; e < n_e; ++e) {
       if (__any_sync(0xffffffffu, s_abort != 0)) break;
-      const int sb = e & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[sb], (e >> 1) & 1))) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&s_full, e & 1))) {
         report(status, MSA_DEV_TIMEOUT);
         s_abort = 1;
         break;
       }
       tc_fence_after();
-      float s[B];
-#pragma unroll
-      for (int c = 0; c < B / 32; ++c) {
-        uint32_t v[32];
-        tc_ld32(lane_base + kColS + sb * 128 + c * 32, v);
-        tc_wait_ld();
-#pragma unroll
-        for (int x = 0; x < 32; ++x) s[c * 32 + x] = __uint_as_float(v[x]);
-      }
-      tc_fence_before();
-      mbar_arrive(&s_free[sb]);
-
       const int2 en = ent[e];
       const int j = en.x;
       const bool sel = row_ok && ((en.y >> ti) & 1);
-      float mx = -INFINITY;
-      if (sel) {
-        const int kmax = t - j * B;  // visible keys: index <= kmax
+      const bool warp_sel = __any_sync(0xffffffffu, sel);
+      const int kmax = t - j * B;  // visible keys: index <= kmax
+      float s[B];
+      if (warp_sel) {
 #pragma unroll
-        for (int c = 0; c < B; ++c) {
-          s[c] = (c <= kmax) ? s[c] * scale_log2 : -INFINITY;
-          mx = fmaxf(mx, s[c]);
+        for (int c = 0; c < B / 32; ++c) {
+          uint32_t v[32];
+          tc_ld32(lane_base + COL_S + c * 32, v);
+#pragma unroll
+          for (int xx = 0; xx < 32; ++xx) s[c * 32 + xx] = __uint_as_float(v[xx]);
+        }
+        tc_wait_ld();
+      }
+      tc_fence_before();
+      mbar_arrive(&s_free);                        // S is in registers: the next S may start
+
+      float mraw = -INFINITY;                      // max of the raw scores
+      if (warp_sel) {
+        if (__any_sync(0xffffffffu, kmax < B - 1)) {
+          // a block that holds some row's own position: mask keys after it
+#pragma unroll
+          for (int c = 0; c < B; ++c) s[c] = (c <= kmax) ? s[c] : -INFINITY;
+        }
+#pragma unroll
+        for (int c = 0; c < B; c += 2) mraw = max3(mraw, s[c], s[c + 1]);
+      }
+      bool rescale = false;
+      float alpha = 1.f;
+      if (sel) {
+        const float mx = mraw * scale_log2;
+        if (m_ref == -INFINITY) {
+          m_ref = mx;                              // first block of this row: O and l are zero
+        } else if (mx > m_ref + kRescaleLog2) {
+          rescale = true;
+          alpha = fast_exp2(m_ref - mx);
+          m_ref = mx;
         }
       }
-      const float m_new = fmaxf(m, mx);
-      const bool rescale = sel && (m != -INFINITY) && (m_new > m);
-      const float alpha = rescale ? fast_exp2(m - m_new) : 1.f;
-      float rs = 0.f;
-      uint32_t pk[B / 2];
-      if (sel) {
-#pragma unroll
-        for (int c = 0; c < B; c += 2) {
-          // l sums the same bf16-rounded weights the P*V product uses, so the
-          // output is an exact convex combination of the rounded weights
-          const uint32_t pp = pack_bf16(fast_exp2(s[c] - m_new), fast_exp2(s[c + 1] - m_new));
-          rs += __uint_as_float(pp << 16) + __uint_as_float(pp & 0xffff0000u);
-          pk[c / 2] = pp;
-        }
-      } else {
-#pragma unroll
-        for (int c = 0; c < B / 2; ++c) pk[c] = 0u;
-      }
-      // previous P*V must be complete before P is overwritten or O rescaled
-      if (e > 0) {
-        if (!__all_sync(0xffffffffu, mbar_wait(&o_done, (e - 1) & 1))) {
+      if (__any_sync(0xffffffffu, rescale)) {
+        // every P*V up to block e-1 must have completed before O is rescaled
+        if (e > 0 && !__all_sync(0xffffffffu, mbar_wait(&o_done[(e - 1) & 1], ((e - 1) >> 1) & 1))) {
           report(status, MSA_DEV_TIMEOUT);
           s_abort = 1;
           break;
         }
         tc_fence_after();
-        if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll
-          for (int c = 0; c < kD / 32; ++c) {
-            uint32_t v[32];
-            tc_ld32(lane_base + kColO + c * 32, v);
-            tc_wait_ld();
+        for (int c = 0; c < kD / 32; ++c) {
+          uint32_t v[32];
+          tc_ld32(lane_base + COL_O + c * 32, v);
+          tc_wait_ld();
 #pragma unroll
-            for (int x = 0; x < 32; ++x) v[x] = __float_as_uint(__uint_as_float(v[x]) * alpha);
-            tc_st32(lane_base + kColO + c * 32, v);
-          }
+          for (int xx = 0; xx < 32; ++xx) v[xx] = __float_as_uint(__uint_as_float(v[xx]) * alpha);
+          tc_st32(lane_base + COL_O + c * 32, v);
         }
+        const float lsum = __uint_as_float((uint32_t)l2) + __uint_as_float((uint32_t)(l2 >> 32));
+        l2 = f2_pack(lsum * alpha, 0.f);
       }
+      // P buffer e&1 was last read by the P*V of block e-2
+      const int pb = e & 1;
+      if (e >= 2 && !__all_sync(0xffffffffu, mbar_wait(&o_done[pb], ((e >> 1) - 1) & 1))) {
+        report(status, MSA_DEV_TIMEOUT);
+        s_abort = 1;
+        break;
+      }
+      tc_fence_after();
+      // P = exp2(s*c - m_ref) rounded to bf16; the row sum adds the same
+      // rounded weights the P*V product uses (exact convex combination)
+      const float m_use = sel ? m_ref : INFINITY;
+      const uint64_t neg_m = f2_pack(-m_use, -m_use);
 #pragma unroll
-      for (int c = 0; c < B / 64; ++c) {
-        uint32_t v[32];
+      for (int cc = 0; cc < B / 64; ++cc) {
+        uint32_t pv[32];
+        if (warp_sel) {
 #pragma unroll
-        for (int x = 0; x < 32; ++x) v[x] = pk[c * 32 + x];
-        tc_st32(lane_base + kColP + c * 32, v);
+          for (int xx = 0; xx < 32; ++xx) {
+            const uint64_t arg = f2_fma(f2_pack(s[64 * cc + 2 * xx], s[64 * cc + 2 * xx + 1]), sl2, neg_m);
+            const uint32_t pp = pack_bf16(fast_exp2(__uint_as_float((uint32_t)arg)),
+                                          fast_exp2(__uint_as_float((uint32_t)(arg >> 32))));
+            l2 = f2_add(l2, ((uint64_t)(pp & 0xffff0000u) << 32) | (uint64_t)(pp << 16));
+            pv[xx] = pp;
+          }
+        } else {
+#pragma unroll
+          for (int xx = 0; xx < 32; ++xx) pv[xx] = 0u;
+        }
+        tc_st32(lane_base + COL_P + pb * 64 + cc * 32, pv);
       }
       tc_wait_st();
       tc_fence_before();
-      mbar_arrive(&p_full);
-      if (sel) {
-        l = l * alpha + rs;
-        m = m_new;
-      }
+      mbar_arrive(&p_full[pb]);
     }
-    // epilogue: O / l -> bf16
+    const float l = __uint_as_float((uint32_t)l2) + __uint_as_float((uint32_t)(l2 >> 32));
+    // epilogue: O / l -> bf16 once the last P*V has completed
     const bool go = !__any_sync(0xffffffffu, s_abort != 0);
-    if (go && __all_sync(0xffffffffu, mbar_wait(&o_done, (n_e - 1) & 1))) {
+    if (go && __all_sync(0xffffffffu, mbar_wait(&o_done[(n_e - 1) & 1], ((n_e - 1) >> 1) & 1))) {
       tc_fence_after();
       const float inv = (l > 0.f) ? 1.f / l : 0.f;
       uint4* dst = reinterpret_cast<uint4*>(
@@ -472,23 +525,23 @@ __global__ void __launch_bounds__(192, 1) prefill_tc_kernel(
 #pragma unroll
       for (int c = 0; c < kD / 32; ++c) {
         uint32_t v[32];
-        tc_ld32(lane_base + kColO + c * 32, v);
+        tc_ld32(lane_base + COL_O + c * 32, v);
         tc_wait_ld();
         if (row_ok) {
 #pragma unroll
-          for (int x = 0; x < 32; x += 8) {
+          for (int xx = 0; xx < 32; xx += 8) {
             uint4 w;
-            w.x = pack_bf16(__uint_as_float(v[x]) * inv, __uint_as_float(v[x + 1]) * inv);
-            w.y = pack_bf16(__uint_as_float(v[x + 2]) * inv, __uint_as_float(v[x + 3]) * inv);
-            w.z = pack_bf16(__uint_as_float(v[x + 4]) * inv, __uint_as_float(v[x + 5]) * inv);
-            w.w = pack_bf16(__uint_as_float(v[x + 6]) * inv, __uint_as_float(v[x + 7]) * inv);
-            dst[(c * 32 + x) / 8] = w;
+            w.x = pack_bf16(__uint_as_float(v[xx]) * inv, __uint_as_float(v[xx + 1]) * inv);
+            w.y = pack_bf16(__uint_as_float(v[xx + 2]) * inv, __uint_as_float(v[xx + 3]) * inv);
+            w.z = pack_bf16(__uint_as_float(v[xx + 4]) * inv, __uint_as_float(v[xx + 5]) * inv);
+            w.w = pack_bf16(__uint_as_float(v[xx + 6]) * inv, __uint_as_float(v[xx + 7]) * inv);
+            dst[(c * 32 + xx) / 8] = w;
           }
         }
       }
       if (row_ok && lse)
         lse[(size_t)(row0 + r_lo + ti) * hq + (size_t)g * G + h] =
-            (l > 0.f) ? (m + log2f(l)) * 0.6931471805599453f : -INFINITY;
+            (l > 0.f) ? (m_ref + log2f(l)) * 0.6931471805599453f : -INFINITY;
     } else if (go) {
       report(status, MSA_DEV_TIMEOUT);
       s_abort = 1;
@@ -505,20 +558,19 @@ __global__ void __launch_bounds__(192, 1) prefill_tc_kernel(
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-int prefill_tile_tokens(int G) { return 128 / G; }
-
-static int plan_tiles(const msa_paged_kv_t* kv, int max_rows, int* tps) {
+// units of one 128-row query tile (128 / G tokens) per CTA
+static int plan_units(const msa_paged_kv_t* kv, int max_rows, int* ups) {
   const int TM = 128 / (kv->num_q_heads / kv->num_kv_heads);
-  *tps = (max_rows + TM - 1) / TM;
-  return kv->batch * (*tps) * kv->num_kv_heads;
+  *ups = (max_rows + TM - 1) / TM;
+  return kv->batch * (*ups) * kv->num_kv_heads;
 }
 
 size_t prefill_ws(const msa_paged_kv_t* kv, int max_rows, int top_k) {
-  int tps;
-  const size_t tiles = plan_tiles(kv, max_rows, &tps);
+  int ups;
+  const size_t units = plan_units(kv, max_rows, &ups);
   const int TM = 128 / (kv->num_q_heads / kv->num_kv_heads);
   const size_t ecap = (size_t)TM * top_k;
-  return tiles * ecap * sizeof(int2) + tiles * sizeof(int) + 256;
+  return units * ecap * sizeof(int2) + units * sizeof(int) + 256;
 }
 
 bool prefill_tc_supported(const msa_paged_kv_t* kv) {
@@ -529,7 +581,7 @@ bool prefill_tc_supported(const msa_paged_kv_t* kv) {
 
 template <int B, int G>
 static cudaError_t launch_tc(const msa_paged_kv_t* kv, const CUtensorMap& tk, const CUtensorMap& tv,
-                             const void* q, const int32_t* cu_q, int tiles, int tps, int ecap,
+                             const void* q, const int32_t* cu_q, int units, int ups, int ecap,
                              const int2* entries, const int* counts, float sl2, void* out,
                              float* lse, cudaStream_t st) {
   constexpr int NST = (B == 128) ? 3 : 4;
@@ -537,9 +589,9 @@ static cudaError_t launch_tc(const msa_paged_kv_t* kv, const CUtensorMap& tk, co
   auto kern = prefill_tc_kernel<B, G>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kern<<<tiles, 192, smem, st>>>(tk, tv, (const bf16*)q, cu_q, kv->page_table, kv->seq_lens,
+  kern<<<units, 192, smem, st>>>(tk, tv, (const bf16*)q, cu_q, kv->page_table, kv->seq_lens,
                                  kv->status_word, kv->num_q_heads, kv->num_kv_heads, kv->num_pages,
-                                 kv->max_blocks_per_seq, tps, ecap, entries, counts, sl2,
+                                 kv->max_blocks_per_seq, ups, ecap, entries, counts, sl2,
                                  (bf16*)out, lse);
   return cudaGetLastError();
 }
@@ -549,14 +601,14 @@ cudaError_t prefill_tc(const msa_paged_kv_t* kv, const void* q, const int32_t* c
                        cudaStream_t st) {
   const int G = kv->num_q_heads / kv->num_kv_heads, B = kv->block_size;
   const int TM = 128 / G;
-  int tps;
-  const int tiles = plan_tiles(kv, max_rows, &tps);
+  int ups;
+  const int units = plan_units(kv, max_rows, &ups);
   const int ecap = TM * top_k;
   int2* entries = (int2*)ws;
-  int* counts = (int*)(entries + (size_t)tiles * ecap);
-  prefill_plan_kernel<<<tiles, 128, 0, st>>>(cu_q, kv->seq_lens, idx, kv->status_word,
+  int* counts = (int*)(entries + (size_t)units * ecap);
+  prefill_plan_kernel<<<units, 128, 0, st>>>(cu_q, kv->seq_lens, idx, kv->status_word,
                                              kv->num_kv_heads, B, kv->max_blocks_per_seq, top_k,
-                                             TM, tps, ecap, entries, counts);
+                                             TM, 1, ups, ecap, entries, counts);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   CUtensorMap tk, tv;
@@ -566,10 +618,10 @@ cudaError_t prefill_tc(const msa_paged_kv_t* kv, const void* q, const int32_t* c
     return cudaErrorInvalidValue;
   const float sl2 = scale * kLog2e;
   if (B == 128)
-    return G == 8 ? launch_tc<128, 8>(kv, tk, tv, q, cu_q, tiles, tps, ecap, entries, counts, sl2, out, lse, st)
-                  : launch_tc<128, 16>(kv, tk, tv, q, cu_q, tiles, tps, ecap, entries, counts, sl2, out, lse, st);
-  return G == 8 ? launch_tc<64, 8>(kv, tk, tv, q, cu_q, tiles, tps, ecap, entries, counts, sl2, out, lse, st)
-                : launch_tc<64, 16>(kv, tk, tv, q, cu_q, tiles, tps, ecap, entries, counts, sl2, out, lse, st);
+    return G == 8 ? launch_tc<128, 8>(kv, tk, tv, q, cu_q, units, ups, ecap, entries, counts, sl2, out, lse, st)
+                  : launch_tc<128, 16>(kv, tk, tv, q, cu_q, units, ups, ecap, entries, counts, sl2, out, lse, st);
+  return G == 8 ? launch_tc<64, 8>(kv, tk, tv, q, cu_q, units, ups, ecap, entries, counts, sl2, out, lse, st)
+                : launch_tc<64, 16>(kv, tk, tv, q, cu_q, units, ups, ecap, entries, counts, sl2, out, lse, st);
 }
 
 }  // namespace msa

@@ -35,14 +35,34 @@ constexpr int kChunk = 64;      // candidates per shared-memory chunk (select_ro
 constexpr int kDecChunk = 128;  // candidates per select_decode pass-1 CTA
 constexpr int kMergeCap = 2048; // keys sorted at once by select_decode pass 2
 
-template <typename T, int D>
-__device__ __forceinline__ void load_qbar(const T* __restrict__ qrow, int G, int g, float* out_i,
-                                          int i) {
-  // qbar[i] = q_{gG}[i] + q_{gG+1}[i] + ... left to right
+// qbar[i..i+VEC) = q_{gG}[i] + q_{gG+1}[i] + ... (left to right over the heads)
+// for VEC = 16 / sizeof(T) consecutive coordinates. All G head loads are
+// issued before the sums, as 16-byte vectors.
+template <typename T>
+__device__ __forceinline__ void load_qbar_vec(const T* __restrict__ qrow, int G, int g, int D, int i,
+                                              float* out) {
+  constexpr int VEC = 16 / sizeof(T);
+  uint4 v[16];
   const T* p = qrow + (size_t)g * G * D + i;
-  float s = to_f32(p[0]);
-  for (int h = 1; h < G; ++h) s = __fadd_rn(s, to_f32(p[(size_t)h * D]));
-  *out_i = s;
+#pragma unroll
+  for (int h = 0; h < 16; ++h)
+    if (h < G) v[h] = *reinterpret_cast<const uint4*>(p + (size_t)h * D);
+  float acc[VEC];
+  {
+    const T* e = reinterpret_cast<const T*>(&v[0]);
+#pragma unroll
+    for (int x = 0; x < VEC; ++x) acc[x] = to_f32(e[x]);
+  }
+#pragma unroll
+  for (int h = 1; h < 16; ++h) {
+    if (h < G) {
+      const T* e = reinterpret_cast<const T*>(&v[h]);
+#pragma unroll
+      for (int x = 0; x < VEC; ++x) acc[x] = __fadd_rn(acc[x], to_f32(e[x]));
+    }
+  }
+#pragma unroll
+  for (int x = 0; x < VEC; ++x) out[x] = acc[x];
 }
 
 // Sorted insertion into a descending list of N keys (L[N-1] smallest).
@@ -115,12 +135,18 @@ __global__ void __launch_bounds__(256) select_rows_kernel(
   const int tid = threadIdx.x;
 
   // qbar for the tile's rows
-  for (int e = tid; e < kRows * D; e += 256) {
-    const int r = e / D, i = e % D;
-    if (r < nr)
-      load_qbar<T, D>(q + (size_t)(row0 + r_lo + r) * hq * D, G, g, &qbar[e], i);
-    else
-      qbar[e] = 0.f;
+  {
+    constexpr int VEC = 16 / sizeof(T);
+    for (int e = tid; e < kRows * (D / VEC); e += 256) {
+      const int r = e / (D / VEC), i = (e % (D / VEC)) * VEC;
+      float* dst = &qbar[r * D + i];
+      if (r < nr) {
+        load_qbar_vec<T>(q + (size_t)(row0 + r_lo + r) * hq * D, G, g, D, i, dst);
+      } else {
+#pragma unroll
+        for (int x = 0; x < VEC; ++x) dst[x] = 0.f;
+      }
+    }
   }
   const int t_first = row_position(L, n_rows, r_lo);
   const int t_last = row_position(L, n_rows, r_lo + nr - 1);
@@ -201,19 +227,39 @@ __global__ void __launch_bounds__(256) select_rows_kernel(
     }
   }
 
-  // merge the SUBS lists of each row into sub 0
+  // merge the SUBS lists of each row pairwise (3 levels). Two descending lists
+  // A, B: max(A[i], B[N-1-i]) holds the top N as a bitonic sequence, which a
+  // half-cleaner network sorts back into descending order.
   uint64_t* my_list = lists + ((size_t)sr * SUBS + ss) * KMAX;
 #pragma unroll
   for (int s = 0; s < KMAX; ++s) my_list[s] = top[s];
   __syncthreads();
-  if (ss == 0 && sr < nr) {
-    for (int o = 1; o < SUBS; ++o) {
-      const uint64_t* other = lists + ((size_t)sr * SUBS + o) * KMAX;
+#pragma unroll
+  for (int w = 1; w < SUBS; w <<= 1) {
+    if ((ss & (2 * w - 1)) == 0) {
+      const uint64_t* other = my_list + (size_t)w * KMAX;
+#pragma unroll
       for (int s = 0; s < KMAX; ++s) {
-        if (other[s] <= top[KMAX - 1]) break;
-        insert_key<KMAX>(top, other[s]);
+        const uint64_t o = other[KMAX - 1 - s];
+        top[s] = top[s] > o ? top[s] : o;
       }
+#pragma unroll
+      for (int stride = KMAX / 2; stride >= 1; stride >>= 1) {
+#pragma unroll
+        for (int s = 0; s < KMAX; ++s) {
+          if ((s & stride) == 0) {
+            const uint64_t a = top[s], c = top[s + stride];
+            top[s] = a > c ? a : c;
+            top[s + stride] = a > c ? c : a;
+          }
+        }
+      }
+#pragma unroll
+      for (int s = 0; s < KMAX; ++s) my_list[s] = top[s];
     }
+    __syncthreads();
+  }
+  if (ss == 0 && sr < nr) {
     const int keep = min(top_k - 1, my_nc);
 #pragma unroll
     for (int s = 0; s < KMAX; ++s) my_list[s] = (s < keep) ? top[s] : 0ull;
@@ -274,7 +320,11 @@ __global__ void __launch_bounds__(kDecChunk) select_decode_pass1(
     return;
   }
   const int tid = threadIdx.x;
-  for (int i = tid; i < D; i += blockDim.x) load_qbar<T, D>(q + (size_t)b * hq * D, G, g, &qbar[i], i);
+  {
+    constexpr int VEC = 16 / sizeof(T);
+    for (int i = tid * VEC; i < D; i += blockDim.x * VEC)
+      load_qbar_vec<T>(q + (size_t)b * hq * D, G, g, D, i, &qbar[i]);
+  }
   {
     int pg = -1;
     if (tid < nc) {
@@ -339,12 +389,13 @@ __global__ void __launch_bounds__(256) select_decode_pass2(
   __syncthreads();
   int head = 0;  // keys already consumed from src
   while (head < total) {
-    const int room = kMergeCap - keep;
-    const int take = min(room, total - head);
-    for (int s = threadIdx.x; s < kMergeCap - keep; s += blockDim.x)
+    const int take = min(kMergeCap - keep, total - head);
+    int n = 1;
+    while (n < keep + take) n <<= 1;  // sort only the next power of two
+    for (int s = threadIdx.x; s < n - keep; s += blockDim.x)
       buf[keep + s] = (s < take) ? src[head + s] : 0ull;
     head += take;
-    bitonic_desc(buf, kMergeCap);
+    bitonic_desc(buf, n);
   }
   for (int s = threadIdx.x; s < 256; s += blockDim.x) chosen[s] = (s < keep) ? buf[s] : 0ull;
   __syncthreads();
