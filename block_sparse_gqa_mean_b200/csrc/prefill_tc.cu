@@ -93,6 +93,13 @@ __device__ __forceinline__ void tc_st32(uint32_t taddr, const uint32_t (&r)[32])
       : "memory");
 }
 
+__device__ __forceinline__ void tc_ld1(uint32_t taddr, uint32_t (&r)[1]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r[0]) : "r"(taddr));
+}
+__device__ __forceinline__ void tc_st1(uint32_t taddr, const uint32_t (&r)[1]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(r[0]) : "memory");
+}
+
 // Shared-memory matrix descriptor, 128-byte swizzle (sm_100 layout: start
 // address, leading and stride byte offsets in 16-byte units, version 1).
 __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
@@ -223,6 +230,35 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
+
+// 2^x for two lanes on the FMA pipe, to share the exponentials with the
+// MUFU unit. x is clamped to [-120, +inf); rint(x) comes from adding
+// 1.5 * 2^23 (the sum's low mantissa bits hold rint(x)), f = x - rint(x) lies
+// in [-0.5, 0.5], 2^f is a cubic minimax fit (relative error 7.5e-5, fitted
+// for this kernel by a Remez exchange on relative error), and rint(x) is
+// added to the exponent field. The result is rounded to bf16 afterwards.
+constexpr uint32_t kMagic = 0x4B400000u;  // 1.5 * 2^23
+__device__ __forceinline__ void exp2_poly_pair(uint64_t arg, float& r0, float& r1) {
+  constexpr uint64_t MAGIC = ((uint64_t)kMagic << 32) | kMagic;
+  constexpr uint64_t NMAGIC = ((uint64_t)(kMagic | 0x80000000u) << 32) | (kMagic | 0x80000000u);
+  constexpr uint64_t NEG1 = 0xBF800000BF800000ull;
+  constexpr uint64_t C0 = 0x3F7FFB49'3F7FFB49ull;   // 9.999280572e-01
+  constexpr uint64_t C1 = 0x3F31798D'3F31798Dull;   // 6.932609677e-01
+  constexpr uint64_t C2 = 0x3E786F0D'3E786F0Dull;   // 2.426111251e-01
+  constexpr uint64_t C3 = 0x3D61FBB0'3D61FBB0ull;   // 5.517166853e-02
+  const float x0 = fmaxf(__uint_as_float((uint32_t)arg), -120.f);
+  const float x1 = fmaxf(__uint_as_float((uint32_t)(arg >> 32)), -120.f);
+  const uint64_t X = f2_pack(x0, x1);
+  const uint64_t T = f2_add(X, MAGIC);
+  const uint64_t J = f2_add(T, NMAGIC);
+  const uint64_t F = f2_fma(J, NEG1, X);
+  uint64_t P = f2_fma(F, C3, C2);
+  P = f2_fma(P, F, C1);
+  P = f2_fma(P, F, C0);
+  r0 = __int_as_float((int)(uint32_t)P + ((int)(uint32_t)T << 23));
+  r1 = __int_as_float((int)(uint32_t)(P >> 32) + ((int)(uint32_t)(T >> 32) << 23));
+}
+
 __device__ __forceinline__ float max3(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
@@ -248,10 +284,14 @@ __global__ void __launch_bounds__(192, 1) prefill_tc_kernel(
   constexpr uint32_t COL_P = 64;   // two P buffers of 64 columns (bf16 pairs)
   constexpr uint32_t COL_S = 192;  // S, 128 columns (fp32)
   constexpr uint32_t COL_O = 320;  // O, 128 columns (fp32)
+  constexpr uint32_t COL_L = 448;  // row sums of P, 16 columns (fp32; column 0 used)
+  constexpr uint32_t IDESC_L = idesc_bf16(128, 16, false);
+  constexpr int ONES = 16 * B * 2; // all-ones B operand [16][B] bf16 for the row sums
 
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  unsigned char* stages = reinterpret_cast<unsigned char*>(
+  unsigned char* ones = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  unsigned char* stages = ones + 4096;
   __shared__ __align__(8) uint64_t kv_full[NST], kv_empty[NST];
   __shared__ __align__(8) uint64_t s_full, s_free, p_full[2], o_done[2], q_ready, fin;
   __shared__ uint32_t s_tmem;
@@ -288,6 +328,9 @@ __global__ void __launch_bounds__(192, 1) prefill_tc_kernel(
     s_abort = 0;
     mbar_fence_init();
   }
+  for (int i = tid; i < ONES / 16; i += blockDim.x)  // bf16 1.0 = 0x3f80
+    reinterpret_cast<uint4*>(ones)[i] = make_uint4(0x3f803f80u, 0x3f803f80u, 0x3f803f80u, 0x3f803f80u);
+  fence_proxy_async_smem();
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(
                      smem_u32(&s_tmem))
@@ -357,11 +400,16 @@ __global__ void __launch_bounds__(192, 1) prefill_tc_kernel(
         if (!mbar_wait(&p_full[pb], (e >> 1) & 1)) { ok = false; break; }
         tc_fence_after();
         const uint32_t vt = smem_u32(stages + (e % NST) * STAGE + TILE);
+        const uint32_t on = smem_u32(ones);
 #pragma unroll
         for (int kk = 0; kk < B / 16; ++kk) {
+          const uint32_t acc = (e > 0 || kk > 0) ? 1u : 0u;
           tc_mma_ts(tmem + COL_O, tmem + COL_P + pb * 64 + kk * 8,
-                    sdesc_sw128(vt + (uint32_t)kk * 2048u, (uint32_t)(TILE / 2), 1024), IDESC_O,
-                    (e > 0 || kk > 0) ? 1u : 0u);
+                    sdesc_sw128(vt + (uint32_t)kk * 2048u, (uint32_t)(TILE / 2), 1024), IDESC_O, acc);
+          // l += P * 1: the same bf16 weights, summed by the same tensor cores
+          tc_mma_ts(tmem + COL_L, tmem + COL_P + pb * 64 + kk * 8,
+                    sdesc_sw128(on + (uint32_t)(kk >> 2) * 2048u + (uint32_t)(kk & 3) * 32u, 16, 1024),
+                    IDESC_L, acc);
         }
         tc_commit(&o_done[pb]);
         tc_commit(&kv_empty[e % NST]);
@@ -409,17 +457,18 @@ __global__ void __launch_bounds__(192, 1) prefill_tc_kernel(
     // has to wait for the P*V in flight. Rows whose token did not select the
     // block use m = +inf, which turns every weight into an exact 0.
     float m_ref = -INFINITY;
-    uint64_t l2 = f2_pack(0.f, 0.f);               // row sum, two fp32 lanes
     const uint64_t sl2 = f2_pack(scale_log2, scale_log2);
+    int2 en_next = ent[0];
     for (int e = 0; e < n_e; ++e) {
       if (__any_sync(0xffffffffu, s_abort != 0)) break;
+      const int2 en = en_next;
+      if (e + 1 < n_e) en_next = ent[e + 1];      // prefetch the next plan entry
       if (!__all_sync(0xffffffffu, mbar_wait(&s_full, e & 1))) {
         report(status, MSA_DEV_TIMEOUT);
         s_abort = 1;
         break;
       }
       tc_fence_after();
-      const int2 en = ent[e];
       const int j = en.x;
       const bool sel = row_ok && ((en.y >> ti) & 1);
       const bool warp_sel = __any_sync(0xffffffffu, sel);
@@ -445,8 +494,13 @@ __global__ void __launch_bounds__(192, 1) prefill_tc_kernel(
 #pragma unroll
           for (int c = 0; c < B; ++c) s[c] = (c <= kmax) ? s[c] : -INFINITY;
         }
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int c = 0; c < B; c += 2) mraw = max3(mraw, s[c], s[c + 1]);
+        for (int c = 0; c < B; c += 8) {
+#pragma unroll
+          for (int a = 0; a < 4; ++a) m4[a] = max3(m4[a], s[c + 2 * a], s[c + 2 * a + 1]);
+        }
+        mraw = max3(m4[0], m4[1], fmaxf(m4[2], m4[3]));
       }
       bool rescale = false;
       float alpha = 1.f;
@@ -477,8 +531,13 @@ __global__ void __launch_bounds__(192, 1) prefill_tc_kernel(
           for (int xx = 0; xx < 32; ++xx) v[xx] = __float_as_uint(__uint_as_float(v[xx]) * alpha);
           tc_st32(lane_base + COL_O + c * 32, v);
         }
-        const float lsum = __uint_as_float((uint32_t)l2) + __uint_as_float((uint32_t)(l2 >> 32));
-        l2 = f2_pack(lsum * alpha, 0.f);
+        {
+          uint32_t lv[1];
+          tc_ld1(lane_base + COL_L, lv);
+          tc_wait_ld();
+          lv[0] = __float_as_uint(__uint_as_float(lv[0]) * alpha);
+          tc_st1(lane_base + COL_L, lv);
+        }
       }
       // P buffer e&1 was last read by the P*V of block e-2
       const int pb = e & 1;
@@ -488,8 +547,8 @@ __global__ void __launch_bounds__(192, 1) prefill_tc_kernel(
         break;
       }
       tc_fence_after();
-      // P = exp2(s*c - m_ref) rounded to bf16; the row sum adds the same
-      // rounded weights the P*V product uses (exact convex combination)
+      // P = exp2(s*c - m_ref) rounded to bf16 (the tensor cores sum the same
+      // rounded weights into l, so the output is an exact convex combination)
       const float m_use = sel ? m_ref : INFINITY;
       const uint64_t neg_m = f2_pack(-m_use, -m_use);
 #pragma unroll
@@ -499,10 +558,14 @@ __global__ void __launch_bounds__(192, 1) prefill_tc_kernel(
 #pragma unroll
           for (int xx = 0; xx < 32; ++xx) {
             const uint64_t arg = f2_fma(f2_pack(s[64 * cc + 2 * xx], s[64 * cc + 2 * xx + 1]), sl2, neg_m);
-            const uint32_t pp = pack_bf16(fast_exp2(__uint_as_float((uint32_t)arg)),
-                                          fast_exp2(__uint_as_float((uint32_t)(arg >> 32))));
-            l2 = f2_add(l2, ((uint64_t)(pp & 0xffff0000u) << 32) | (uint64_t)(pp << 16));
-            pv[xx] = pp;
+            if (xx & 1) {  // every other pair on the FMA pipe, the rest on MUFU
+              float p0, p1;
+              exp2_poly_pair(arg, p0, p1);
+              pv[xx] = pack_bf16(p0, p1);
+            } else {
+              pv[xx] = pack_bf16(fast_exp2(__uint_as_float((uint32_t)arg)),
+                                 fast_exp2(__uint_as_float((uint32_t)(arg >> 32))));
+            }
           }
         } else {
 #pragma unroll
@@ -514,11 +577,17 @@ __global__ void __launch_bounds__(192, 1) prefill_tc_kernel(
       tc_fence_before();
       mbar_arrive(&p_full[pb]);
     }
-    const float l = __uint_as_float((uint32_t)l2) + __uint_as_float((uint32_t)(l2 >> 32));
     // epilogue: O / l -> bf16 once the last P*V has completed
     const bool go = !__any_sync(0xffffffffu, s_abort != 0);
     if (go && __all_sync(0xffffffffu, mbar_wait(&o_done[(n_e - 1) & 1], ((n_e - 1) >> 1) & 1))) {
       tc_fence_after();
+      float l;
+      {
+        uint32_t lv[1];
+        tc_ld1(lane_base + COL_L, lv);
+        tc_wait_ld();
+        l = __uint_as_float(lv[0]);
+      }
       const float inv = (l > 0.f) ? 1.f / l : 0.f;
       uint4* dst = reinterpret_cast<uint4*>(
           out + ((size_t)(row0 + r_lo + ti) * hq + (size_t)g * G + h) * kD);
@@ -585,7 +654,7 @@ static cudaError_t launch_tc(const msa_paged_kv_t* kv, const CUtensorMap& tk, co
                              const int2* entries, const int* counts, float sl2, void* out,
                              float* lse, cudaStream_t st) {
   constexpr int NST = (B == 128) ? 3 : 4;
-  const size_t smem = (size_t)NST * 2 * B * kD * 2 + 1024;
+  const size_t smem = 4096 + (size_t)NST * 2 * B * kD * 2 + 1024;
   auto kern = prefill_tc_kernel<B, G>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
