@@ -13,9 +13,12 @@ The default workload is the prefill one (batch 1, 32768 tokens, 32/4 heads,
 d 128, block 128, top-k 16); a paged-decode block (batch 32, 131072 cached
 tokens, 32/8 heads, block 64, top-k 32) is measured in the same run.
 
-Timing: W untimed warm-up steps, then K steps between a barrier and
-torch.cuda.synchronize() on both sides, CUDA events on the launching stream,
-max over ranks. Inputs of every step exceed the 126 MB L2 (prefill: 0.7 GB;
+Timing: W untimed warm-up steps; the step is then captured in a CUDA graph
+(the library never allocates or synchronises) and K replays are timed between
+a barrier and torch.cuda.synchronize() on both sides, with CUDA events on the
+replay stream, max over ranks. Per-call times come from graphs of each call
+alone. The end-to-end figure runs the public Python calls eagerly, with the
+step's host-to-device and device-to-host copies inside the timed region. Inputs of every step exceed the 126 MB L2 (prefill: 0.7 GB;
 paged decode: ~0.53 GB read per step); the 1M-context decode working set
 (~42 MB) does not, so that workload writes a 256 MB buffer between steps.
 Under torchrun each rank runs its own replica of the workload (independent
@@ -156,6 +159,38 @@ def max_over_ranks(x: float, world: int) -> float:
     return float(t.item())
 
 
+def capture_graph(fn):
+    """CUDA graph of fn's launches (the library allocates nothing and never
+    synchronises, so every call can be captured)."""
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        fn()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    torch.cuda.synchronize()
+    return g
+
+
+def time_graph(g, steps, before=None):
+    """Mean device time of one replay (CUDA events on the replay stream).
+    `before(i)` runs untimed work (an L2 flush) ahead of replay i."""
+    stream = torch.cuda.current_stream()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    for i in range(steps):
+        if before is not None:
+            before(i)
+        ev[i][0].record(stream)
+        g.replay()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    return sum(a.elapsed_time(b) for a, b in ev) / steps
+
+
 def attended_pairs(T: int, B: int, k: int) -> int:
     """Query-key pairs per head of a full causal prefill: row t sees its own
     block up to t plus k-1 complete past blocks (all of them when fewer)."""
@@ -188,36 +223,36 @@ def run_prefill(w, steps, warmup, world):
                          dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
-    def step(ev=None):
-        if ev: ev[0].record(stream)
+    def do_append():
         msa.build_block_cache(cache, k_new, v_new, cu, T)
-        if ev: ev[1].record(stream)
+
+    def do_select():
         msa.select_topk(cache, q, w.top_k, cu_q=cu, max_rows_per_seq=T, block_idx=idx,
                         workspace=ws_sel)
-        if ev: ev[2].record(stream)
+
+    def do_attn():
         msa.sparse_attn_prefill(cache, q, idx, cu_q=cu, max_rows_per_seq=T, out=out, lse=lse,
                                 workspace=ws_att)
-        if ev: ev[3].record(stream)
+
+    def step():
+        do_append()
+        do_select()
+        do_attn()
 
     for _ in range(warmup):
         step()
     torch.cuda.synchronize()
     if cache.device_status() != 0:
         raise RuntimeError(f"device status {cache.device_status():#x}")
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    g_step = capture_graph(step)
+    g_ops = [capture_graph(f) for f in (do_append, do_select, do_attn)]
     barrier(world)
     torch.cuda.synchronize()
     with Clocks(torch.cuda.current_device()) as clk:
-        t0 = torch.cuda.Event(enable_timing=True)
-        t1 = torch.cuda.Event(enable_timing=True)
-        t0.record(stream)
-        for i in range(steps):
-            step(evs[i])
-        t1.record(stream)
-        torch.cuda.synchronize()
+        step_ms = time_graph(g_step, steps)
     barrier(world)
-    total_ms = t0.elapsed_time(t1)
-    k_ms = [sum(e[i].elapsed_time(e[i + 1]) for e in evs) / steps for i in range(3)]
+    k_ms = [time_graph(gg, steps) for gg in g_ops]
+    total_ms = step_ms * steps
 
     # executed (union) tile-blocks of the tensor-core schedule, for context
     G = w.group
@@ -328,30 +363,33 @@ def run_decode(w, steps, warmup, world, flush_l2):
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev) if flush_l2 else None
     stream = torch.cuda.current_stream()
 
-    def step(ev=None):
-        if ev: ev[0].record(stream)
+    def do_append():
         msa.build_block_cache(cache, kn, vn, cu, 1)
-        if ev: ev[1].record(stream)
+
+    def do_select():
         msa.select_topk(cache, q, w.top_k, block_idx=idx, workspace=ws_sel)
-        if ev: ev[2].record(stream)
+
+    def do_attn():
         msa.sparse_attn_decode(cache, q, idx, out=out, lse=lse, workspace=ws_dec)
-        if ev: ev[3].record(stream)
+
+    def step():
+        do_append()
+        do_select()
+        do_attn()
 
     for _ in range(warmup):
         step()
     torch.cuda.synchronize()
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    g_step = capture_graph(step)
+    g_ops = [capture_graph(f) for f in (do_append, do_select, do_attn)]
+    flush_fn = (lambda i: flush.fill_(i & 0xFF)) if flush is not None else None
     barrier(world)
     torch.cuda.synchronize()
     with Clocks(torch.cuda.current_device()) as clk:
-        for i in range(steps):
-            if flush is not None:
-                flush.fill_(i & 0xFF)
-            step(evs[i])
-        torch.cuda.synchronize()
+        step_ms = time_graph(g_step, steps, flush_fn)
     barrier(world)
-    per_step = [e[0].elapsed_time(e[3]) for e in evs]
-    k_ms = [sum(e[i].elapsed_time(e[i + 1]) for e in evs) / steps for i in range(3)]
+    k_ms = [time_graph(gg, steps, flush_fn) for gg in g_ops]
+    per_step = [step_ms]
 
     # end to end: q and the new K/V rows from pinned host memory, out back to host
     hq_, hk, hv = q.cpu().pin_memory(), kn.cpu().pin_memory(), vn.cpu().pin_memory()
@@ -383,7 +421,7 @@ def run_decode(w, steps, warmup, world, flush_l2):
     status = cache.device_status()
     if status != 0:
         raise RuntimeError(f"device status {status:#x}")
-    return {"step_ms": sum(per_step) / steps, "kernel_ms": k_ms, "clocks": clk.summary(),
+    return {"step_ms": per_step[0], "kernel_ms": k_ms, "clocks": clk.summary(),
             "e2e_ms": e2e_ms, "h2d": (hq_.numel() + hk.numel() + hv.numel()) * 2,
             "d2h": hout.numel() * 2, "launches_per_step": 1 + 2 + 2}
 

@@ -321,8 +321,8 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const float* __rest
 // host side
 // ---------------------------------------------------------------------------
 int decode_splits(const msa_paged_kv_t* kv, int top_k, int num_sms) {
-  // several CTAs per SM (two-stage pipelines of 32-64 KB each) over several
-  // waves, so the HBM stream has enough bytes in flight and a small tail
+  // about eight CTAs per SM over the whole grid (three resident at a time),
+  // so the HBM stream has bytes in flight and the last wave is short
   const int units = kv->batch * kv->num_kv_heads;
   int splits = (8 * num_sms + units - 1) / units;
   if (splits > top_k) splits = top_k;

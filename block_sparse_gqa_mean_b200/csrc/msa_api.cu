@@ -14,6 +14,7 @@ cudaError_t append_pool(const msa_paged_kv_t*, const void*, const void*, const i
 cudaError_t select_rows(const msa_paged_kv_t*, const void*, const int32_t*, int, int, int32_t*,
                         float*, cudaStream_t);
 bool select_rows_supported(int top_k);
+bool select_decode_supported(const msa_paged_kv_t*);
 size_t select_decode_ws(const msa_paged_kv_t*, int top_k);
 cudaError_t select_decode(const msa_paged_kv_t*, const void*, int, int32_t*, float*, void*,
                           cudaStream_t);
@@ -161,6 +162,7 @@ msa_status_t msa_select_topk(const msa_paged_kv_t* kv, const void* q, const int3
   cudaStream_t st = (cudaStream_t)stream;
   if (!cu_q) {
     if (num_rows != kv->batch) return MSA_ERR_INVALID_ARG;
+    if (!select_decode_supported(kv)) return MSA_ERR_UNSUPPORTED;
     const size_t need = select_decode_ws(kv, top_k);
     if (workspace_bytes < need || (need && (!workspace || !aligned(workspace, 16))))
       return MSA_ERR_WORKSPACE;

@@ -21,9 +21,10 @@
 //                    micro-kernel and keeps per-thread sorted top lists that
 //                    are merged at the end.
 //  * select_decode - one row per sequence with thousands of candidates. Pass 1
-//                    splits the candidates into chunks of 128 across CTAs
+//                    splits the candidates into chunks of 64 across CTAs
 //                    (thread per candidate, bitonic sort of the chunk in shared
-//                    memory, keep k-1); pass 2 merges the chunk lists.
+//                    memory, keep k-1); pass 2 merges the sorted chunk lists
+//                    with a warp-wide tournament.
 #include "common.cuh"
 
 namespace msa {
@@ -32,8 +33,8 @@ namespace {
 
 constexpr int kRows = 32;       // rows per select_rows CTA
 constexpr int kChunk = 64;      // candidates per shared-memory chunk (select_rows)
-constexpr int kDecChunk = 128;  // candidates per select_decode pass-1 CTA
-constexpr int kMergeCap = 2048; // keys sorted at once by select_decode pass 2
+constexpr int kDecChunk = 64;   // candidates per select_decode pass-1 CTA
+constexpr int kMaxChunksPerLane = 8;  // pass 2: chunk lists per lane (256 chunks)
 
 // qbar[i..i+VEC) = q_{gG}[i] + q_{gG+1}[i] + ... (left to right over the heads)
 // for VEC = 16 / sizeof(T) consecutive coordinates. All G head loads are
@@ -368,13 +369,17 @@ __global__ void __launch_bounds__(kDecChunk) select_decode_pass1(
   for (int s = tid; s < kw; s += blockDim.x) out[s] = keys[s];
 }
 
-__global__ void __launch_bounds__(256) select_decode_pass2(
+// Pass 2: one warp per (sequence, group) merges the chunk lists, each already
+// sorted by pass 1, with a tournament: every round the lanes offer the heads
+// of their chunks, the warp maximum is taken and its chunk advances.
+__global__ void __launch_bounds__(32) select_decode_pass2(
     const uint64_t* __restrict__ ws, const int32_t* __restrict__ seq_lens, int hkv, int B,
     int max_blocks, int kw, int nchunks, int top_k, int32_t* __restrict__ idx,
     float* __restrict__ score) {
-  __shared__ uint64_t buf[kMergeCap];
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  uint64_t* lists = reinterpret_cast<uint64_t*>(smem_raw);  // [nch][kw]
   __shared__ uint64_t chosen[256];
-  const int g = blockIdx.x, b = blockIdx.y;
+  const int g = blockIdx.x, b = blockIdx.y, lane = threadIdx.x;
   const int L = seq_lens[b];
   const size_t outo = ((size_t)b * hkv + g) * top_k;
   if (L < 1 || L > max_blocks * B) return;  // reported by pass 1
@@ -384,41 +389,70 @@ __global__ void __launch_bounds__(256) select_decode_pass2(
   const int nch = (ncand + kDecChunk - 1) / kDecChunk;
   const uint64_t* src = ws + ((size_t)b * hkv + g) * nchunks * kw;
   const int total = nch * kw;
-  // running top list lives in buf[0 .. keep); append batches behind it, sort, keep
-  for (int s = threadIdx.x; s < kMergeCap; s += blockDim.x) buf[s] = 0ull;
-  __syncthreads();
-  int head = 0;  // keys already consumed from src
-  while (head < total) {
-    const int take = min(kMergeCap - keep, total - head);
-    int n = 1;
-    while (n < keep + take) n <<= 1;  // sort only the next power of two
-    for (int s = threadIdx.x; s < n - keep; s += blockDim.x)
-      buf[keep + s] = (s < take) ? src[head + s] : 0ull;
-    head += take;
-    bitonic_desc(buf, n);
+  for (int i0 = 0; i0 < total; i0 += 8 * 32) {  // eight independent loads per lane in flight
+    uint64_t v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = i0 + u * 32 + lane;
+      v[u] = i < total ? src[i] : 0ull;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = i0 + u * 32 + lane;
+      if (i < total) lists[i] = v[u];
+    }
   }
-  for (int s = threadIdx.x; s < 256; s += blockDim.x) chosen[s] = (s < keep) ? buf[s] : 0ull;
-  __syncthreads();
-  // ascending output: rank by block index (keep <= 255)
-  for (int a = threadIdx.x; a < keep; a += blockDim.x) {
+  __syncwarp();
+  int ptr[kMaxChunksPerLane];
+  uint64_t head[kMaxChunksPerLane];
+#pragma unroll
+  for (int s = 0; s < kMaxChunksPerLane; ++s) {
+    const int c = lane + 32 * s;
+    ptr[s] = 0;
+    head[s] = (c < nch) ? lists[(size_t)c * kw] : 0ull;
+  }
+  int cnt = 0;
+  for (; cnt < keep; ++cnt) {
+    uint64_t best = 0ull;
+#pragma unroll
+    for (int s = 0; s < kMaxChunksPerLane; ++s) best = head[s] > best ? head[s] : best;
+    uint64_t wb = best;
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+      const uint32_t lo = __shfl_xor_sync(0xffffffffu, (uint32_t)wb, o);
+      const uint32_t hi = __shfl_xor_sync(0xffffffffu, (uint32_t)(wb >> 32), o);
+      const uint64_t other = ((uint64_t)hi << 32) | lo;
+      wb = other > wb ? other : wb;
+    }
+    if (wb == 0ull) break;  // fewer real candidates than requested (bad pages)
+#pragma unroll
+    for (int s = 0; s < kMaxChunksPerLane; ++s) {
+      if (head[s] == wb) {  // keys are unique: exactly one lane, one chunk
+        const int c = lane + 32 * s;
+        const int nxt = ++ptr[s];
+        head[s] = (nxt < kw) ? lists[(size_t)c * kw + nxt] : 0ull;
+      }
+    }
+    if (lane == 0) chosen[cnt] = wb;
+  }
+  __syncwarp();
+  // ascending output: rank by block index
+  for (int a = lane; a < cnt; a += 32) {
     const uint64_t ka = chosen[a];
-    if (ka == 0ull) continue;
     const int ja = key_block(ka);
     int rank = 0;
-    for (int c2 = 0; c2 < keep; ++c2)
-      if (chosen[c2] != 0ull && key_block(chosen[c2]) < ja) ++rank;
+    for (int c2 = 0; c2 < cnt; ++c2)
+      if (key_block(chosen[c2]) < ja) ++rank;
     idx[outo + rank] = ja;
     if (score) score[outo + rank] = key_score(ka);
   }
-  if (threadIdx.x == 0) {
-    int cnt = 0;
-    for (int a = 0; a < keep; ++a) cnt += chosen[a] != 0ull;
+  if (lane == 0) {
     idx[outo + cnt] = own;
     if (score) score[outo + cnt] = __int_as_float(0x7f800000);
-    for (int s = cnt + 1; s < top_k; ++s) {
-      idx[outo + s] = -1;
-      if (score) score[outo + s] = __int_as_float(0xff800000);
-    }
+  }
+  for (int s = cnt + 1 + lane; s < top_k; s += 32) {
+    idx[outo + s] = -1;
+    if (score) score[outo + s] = __int_as_float(0xff800000);
   }
 }
 
@@ -471,6 +505,12 @@ cudaError_t select_rows(const msa_paged_kv_t* kv, const void* q, const int32_t* 
 
 bool select_rows_supported(int top_k) { return top_k - 1 <= 64; }
 
+// decode selection merges at most 32 * kMaxChunksPerLane chunk lists of
+// kDecChunk candidates
+bool select_decode_supported(const msa_paged_kv_t* kv) {
+  return kv->max_blocks_per_seq <= 32 * kMaxChunksPerLane * kDecChunk;
+}
+
 static int decode_nchunks(const msa_paged_kv_t* kv) {
   return (kv->max_blocks_per_seq + kDecChunk - 1) / kDecChunk;
 }
@@ -496,7 +536,11 @@ static cudaError_t launch_decode_sel(const msa_paged_kv_t* kv, const void* q, in
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   dim3 g2(kv->num_kv_heads, kv->batch);
-  select_decode_pass2<<<g2, 256, 0, st>>>((const uint64_t*)ws, kv->seq_lens, kv->num_kv_heads,
+  const size_t smem2 = (size_t)nch * kw * 8;
+  e = cudaFuncSetAttribute(select_decode_pass2, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem2);
+  if (e != cudaSuccess) return e;
+  select_decode_pass2<<<g2, 32, smem2, st>>>((const uint64_t*)ws, kv->seq_lens, kv->num_kv_heads,
                                           kv->block_size, kv->max_blocks_per_seq, kw, nch, top_k,
                                           idx, score);
   return cudaGetLastError();

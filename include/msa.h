@@ -37,7 +37,8 @@
  *    reads the status word after synchronising and clears it when it wishes.
  *  - Supported shapes: head_dim 64 or 128; block_size 64 or 128;
  *    G = num_q_heads / num_kv_heads an integer in 1..16; 1 <= top_k <= 256.
- *    bf16 attention needs head_dim 128; bf16 prefill attention needs G 8 or 16.
+ *    bf16 attention needs head_dim 128; bf16 prefill attention needs G 8 or 16;
+ *    decode selection (cu_q == NULL) needs max_blocks_per_seq <= 16384.
  *
  * Memory layout (all row-major)
  *  - K/V pages       : [num_pages][num_kv_heads][block_size][head_dim], dtype
