@@ -473,6 +473,8 @@ def main():
     ap.add_argument("--oracle-rows", type=int, default=256)
     ap.add_argument("--seq-len", type=int, default=0,
                     help="override the prefill length (profiling of a smaller case)")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="override the decode batch (profiling of a smaller case)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -480,6 +482,8 @@ def main():
     w = workloads.ALL[args.workload]()
     if args.seq_len and w.kind == "prefill":
         w = workloads.ALL[args.workload](ctx=(args.seq_len,))
+    if args.batch and w.kind == "decode" and w.name != "decode_1m_bf16":
+        w = workloads.ALL[args.workload](batch=args.batch)
     pk = peaks()
 
     if args.impl == "reference":
