@@ -23,6 +23,7 @@ __global__ void __launch_bounds__(128) append_pool_kernel(
     T* __restrict__ k_pages, T* __restrict__ v_pages, float* __restrict__ centroids,
     const int32_t* __restrict__ page_table, const int32_t* __restrict__ seq_lens,
     uint32_t* status, int hkv, int B, int num_pages, int max_blocks) {
+  pdl_wait();
   const int lb = blockIdx.x;  // local block index among the blocks this append touches
   const int b = blockIdx.y;
   const int g = blockIdx.z;
@@ -74,6 +75,7 @@ __global__ void __launch_bounds__(128) append_pool_kernel(
     for (int u = 0; u < n; ++u) s = __fadd_rn(s, to_f32(tile[u * D + i]));
     centroids[((size_t)page * hkv + g) * D + i] = __fdiv_rn(s, (float)n);
   }
+  pdl_release();
 }
 
 template <typename T, int D>
@@ -85,11 +87,10 @@ static cudaError_t launch_append(const msa_paged_kv_t* kv, const void* k_new, co
   cudaError_t e = cudaFuncSetAttribute(append_pool_kernel<T, D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  append_pool_kernel<T, D><<<grid, 128, smem, st>>>(
-      (const T*)k_new, (const T*)v_new, cu_new, (T*)kv->k_pages, (T*)kv->v_pages, kv->centroids,
-      kv->page_table, kv->seq_lens, kv->status_word, kv->num_kv_heads, B, kv->num_pages,
-      kv->max_blocks_per_seq);
-  return cudaGetLastError();
+  return launch_pdl(append_pool_kernel<T, D>, grid, dim3(128), smem, st, (const T*)k_new,
+                    (const T*)v_new, cu_new, (T*)kv->k_pages, (T*)kv->v_pages, kv->centroids,
+                    (const int32_t*)kv->page_table, (const int32_t*)kv->seq_lens, kv->status_word,
+                    kv->num_kv_heads, B, kv->num_pages, kv->max_blocks_per_seq);
 }
 
 cudaError_t append_pool(const msa_paged_kv_t* kv, const void* k_new, const void* v_new,

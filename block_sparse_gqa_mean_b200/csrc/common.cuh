@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "msa.h"
 
 namespace msa {
@@ -16,6 +18,34 @@ typedef __nv_bfloat16 bf16;
 // hundred ns per poll this is well above any legitimate wait and well below a
 // second, after which the kernel records MSA_DEV_TIMEOUT and unwinds.
 constexpr uint32_t kSpinLimit = 1u << 22;
+
+// Programmatic dependent launch. A kernel launched with launch_pdl may begin
+// while its predecessor on the stream is still running: it calls pdl_wait()
+// before it touches global memory (which returns once the predecessor has
+// completed and its writes are visible) and pdl_release() once its last
+// global write is done, which lets its successor launch as the CTAs drain
+// (released earlier, waiting successor CTAs were measured to slow the running
+// kernel). Both are no-ops for an ordinary launch.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_release() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... P, typename... A>
+inline cudaError_t launch_pdl(void (*kernel)(P...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t st, A&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<A>(args)...);
+}
 
 __device__ __forceinline__ void report(uint32_t* status, uint32_t bits) {
   if (status) atomicOr(status, bits);

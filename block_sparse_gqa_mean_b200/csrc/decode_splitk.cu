@@ -82,6 +82,7 @@ __global__ void __launch_bounds__(128) decode_splitk_kernel(
   __shared__ int s_n;
   __shared__ int s_abort;
 
+  pdl_wait();
   const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int G = hq / hkv;
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
@@ -293,6 +294,7 @@ __global__ void __launch_bounds__(128) decode_splitk_kernel(
     ws_o[part * kD + tid] = lsum > 0.f ? acc / lsum : 0.f;
     if (tid == 0) ws_lse[part] = lsum > 0.f ? M + log2f(lsum) : -INFINITY;
   }
+  pdl_release();
 }
 
 // Merge the split partials of each (sequence, head) by log-sum-exp.
@@ -301,6 +303,7 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const float* __rest
                                                              const float* __restrict__ ws_lse,
                                                              int splits, T* __restrict__ out,
                                                              float* __restrict__ lse) {
+  pdl_wait();
   const size_t bh = blockIdx.x;
   const int tid = threadIdx.x;
   float M = -INFINITY;
@@ -315,6 +318,7 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const float* __rest
   }
   out[bh * kD + tid] = from_f32<T>(w > 0.f ? acc / w : 0.f);
   if (lse && tid == 0) lse[bh] = (M + log2f(w)) * 0.6931471805599453f;
+  pdl_release();
 }
 
 // ---------------------------------------------------------------------------
@@ -363,24 +367,22 @@ cudaError_t decode_splitk(const msa_paged_kv_t* kv, const void* q, const int32_t
     e = cudaFuncSetAttribute(decode_splitk_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem);
     if (e != cudaSuccess) return e;
-    decode_splitk_kernel<64><<<grid, 128, smem, st>>>(
-        tk, tv, (const bf16*)q, idx, kv->page_table, kv->seq_lens, kv->status_word, top_k,
-        kv->num_q_heads, kv->num_kv_heads, kv->num_pages, kv->max_blocks_per_seq, sl2, splits, per,
-        ws_o, ws_lse);
+    e = launch_pdl(decode_splitk_kernel<64>, grid, dim3(128), smem, st, tk, tv, (const bf16*)q,
+                   idx, (const int32_t*)kv->page_table, (const int32_t*)kv->seq_lens,
+                   kv->status_word, top_k, kv->num_q_heads, kv->num_kv_heads, kv->num_pages,
+                   kv->max_blocks_per_seq, sl2, splits, per, ws_o, ws_lse);
   } else {
     e = cudaFuncSetAttribute(decode_splitk_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem);
     if (e != cudaSuccess) return e;
-    decode_splitk_kernel<128><<<grid, 128, smem, st>>>(
-        tk, tv, (const bf16*)q, idx, kv->page_table, kv->seq_lens, kv->status_word, top_k,
-        kv->num_q_heads, kv->num_kv_heads, kv->num_pages, kv->max_blocks_per_seq, sl2, splits, per,
-        ws_o, ws_lse);
+    e = launch_pdl(decode_splitk_kernel<128>, grid, dim3(128), smem, st, tk, tv, (const bf16*)q,
+                   idx, (const int32_t*)kv->page_table, (const int32_t*)kv->seq_lens,
+                   kv->status_word, top_k, kv->num_q_heads, kv->num_kv_heads, kv->num_pages,
+                   kv->max_blocks_per_seq, sl2, splits, per, ws_o, ws_lse);
   }
-  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  decode_combine_kernel<bf16><<<kv->batch * kv->num_q_heads, 128, 0, st>>>(ws_o, ws_lse, splits,
-                                                                          (bf16*)out, lse);
-  return cudaGetLastError();
+  return launch_pdl(decode_combine_kernel<bf16>, dim3(kv->batch * kv->num_q_heads), dim3(128), 0,
+                    st, (const float*)ws_o, (const float*)ws_lse, splits, (bf16*)out, lse);
 }
 
 }  // namespace msa

@@ -21,11 +21,19 @@
 //                    micro-kernel and keeps per-thread sorted top lists that
 //                    are merged at the end.
 //  * select_decode - one row per sequence with thousands of candidates. Pass 1
-//                    splits the candidates into chunks of 64 across CTAs
-//                    (thread per candidate, bitonic sort of the chunk in shared
-//                    memory, keep k-1); pass 2 merges the sorted chunk lists
-//                    with a warp-wide tournament.
+//                    cuts the candidates into chunks of 64 and streams whole
+//                    pages of the block cache (every group of a candidate in
+//                    one bulk copy) through persistent CTAs with a producer
+//                    warp, thread per (candidate, group), a register bitonic
+//                    sort per group and chunk, keep k-1; pass 2 merges the
+//                    sorted chunk lists with a warp-wide tournament.
+#include <algorithm>
+#include <map>
+#include <mutex>
+#include <tuple>
+
 #include "common.cuh"
+#include "tma.cuh"
 
 namespace msa {
 
@@ -35,6 +43,19 @@ constexpr int kRows = 32;       // rows per select_rows CTA
 constexpr int kChunk = 64;      // candidates per shared-memory chunk (select_rows)
 constexpr int kDecChunk = 64;   // candidates per select_decode pass-1 CTA
 constexpr int kMaxChunksPerLane = 8;  // pass 2: chunk lists per lane (256 chunks)
+constexpr int kPass1Threads = 128;  // decode pass 1: consumer threads (plus one producer warp)
+
+// decode pass 1: candidates per step, a power of two <= 32 with SC * hkv <= 128
+__host__ __device__ inline int pass1_sc(int hkv) {
+  int sc = 32;
+  while (sc > 1 && sc * hkv > kPass1Threads) sc >>= 1;
+  return sc;
+}
+// one stage: SC padded page copies, then the item's qbar rows; 128-byte multiple
+__host__ __device__ inline int pass1_stage_bytes(int hkv, int D) {
+  const int page = hkv * D * 4;
+  return (pass1_sc(hkv) * (page + 16) + page + 127) & ~127;
+}
 
 // qbar[i..i+VEC) = q_{gG}[i] + q_{gG+1}[i] + ... (left to right over the heads)
 // for VEC = 16 / sizeof(T) consecutive coordinates. All G head loads are
@@ -114,7 +135,7 @@ __global__ void __launch_bounds__(256) select_rows_kernel(
     float* __restrict__ score) {
   constexpr int SUBS = 256 / kRows;  // 8 threads per row in the selection phase
   constexpr int CP = D + 4;          // padded centroid row (bank spread)
-  extern __shared__ __align__(16) unsigned char smem_raw[];
+  extern __shared__ __align__(128) unsigned char smem_raw[];
   float* qbar = reinterpret_cast<float*>(smem_raw);                  // [kRows][D]
   float* cent = qbar + kRows * D;                                     // [kChunk][CP]
   float* sc = cent + kChunk * CP;                                     // [kRows][kChunk]
@@ -272,113 +293,394 @@ __global__ void __launch_bounds__(256) select_rows_kernel(
 // ---------------------------------------------------------------------------
 // select_decode
 // ---------------------------------------------------------------------------
-// Bitonic sort of n (power of two) keys in shared memory, descending.
-__device__ void bitonic_desc(uint64_t* k, int n) {
-  for (int size = 2; size <= n; size <<= 1) {
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      __syncthreads();
-      for (int t = threadIdx.x; t < n / 2; t += blockDim.x) {
-        const int lo = 2 * t - (t & (stride - 1));
-        const int hi = lo + stride;
-        const bool desc = ((lo & size) == 0);
-        const uint64_t a = k[lo], c = k[hi];
-        if (desc ? (a < c) : (a > c)) {
-          k[lo] = c;
-          k[hi] = a;
+// qbar of every (sequence, group) for decode: the group's query heads summed
+// left to right in fp32, the same order load_qbar_vec uses. [batch][hkv][D].
+// One CTA per (group, sequence), one thread per coordinate, all head loads in
+// flight together.
+template <typename T, int D>
+__global__ void __launch_bounds__(D) select_decode_qbar(const T* __restrict__ q, int hq, int hkv,
+                                                       float* __restrict__ qbar,
+                                                       unsigned int* __restrict__ next_item) {
+  pdl_wait();
+  const int g = blockIdx.x, b = blockIdx.y, i = threadIdx.x;
+  if (g == 0 && b == 0 && i == 0) *next_item = 0u;  // pass 1's work counter
+  const int G = hq / hkv;
+  const T* p = q + ((size_t)b * hq + (size_t)g * G) * D + i;
+  float v[16];
+#pragma unroll
+  for (int h = 0; h < 16; ++h) v[h] = h < G ? to_f32(p[(size_t)h * D]) : 0.f;
+  float a = v[0];
+#pragma unroll
+  for (int h = 1; h < 16; ++h)
+    if (h < G) a = __fadd_rn(a, v[h]);
+  qbar[((size_t)b * hkv + g) * D + i] = a;
+  pdl_release();
+}
+
+__device__ __forceinline__ uint64_t shfl_xor_u64(uint64_t v, int m) {
+  const uint32_t lo = __shfl_xor_sync(0xffffffffu, (uint32_t)v, m);
+  const uint32_t hi = __shfl_xor_sync(0xffffffffu, (uint32_t)(v >> 32), m);
+  return ((uint64_t)hi << 32) | lo;
+}
+
+// Pass 1 of decode selection. An item is (sequence b, chunk c of 64 candidate
+// blocks, subset gs of hg consecutive KV groups); items are numbered over the
+// non-empty chunks and claimed by persistent CTAs from a counter that the
+// qbar kernel zeroes, so faster CTAs take more items. The block cache
+// keeps all groups of a page together, so one bulk copy brings one candidate
+// for the item's hg groups (hg * D fp32, 2 KB for 4 groups of d 128). An item
+// is streamed in KPL steps of SC = 64 / KPL candidates through an NST-stage
+// ring of shared memory.
+//   * warp 4 (producer) reads the page-table entries one step ahead, and per
+//     step issues the page copies plus a copy of the item's qbar rows, all
+//     completing on the stage's `full` mbarrier;
+//   * warps 0-3 (consumers): thread t scores candidate t % SC of the step for
+//     group gs * hg + t / SC with the canonical fp32 fma chain, keeps the key in
+//     register slot `step`, and the warp releases the stage on `empty`. After
+//     the item's last step the SC lanes of a group hold its 64 keys (KPL
+//     each) and sort them with a bitonic network (in-register strides below
+//     KPL, shuffles above); element e of the sorted order is rank e.
+template <int D, int KPL, int NST>
+__global__ void __launch_bounds__(kPass1Threads + 32, 1) select_decode_pass1(
+    const float* __restrict__ qbar_all, const float* __restrict__ centroids,
+    const int32_t* __restrict__ page_table, const int32_t* __restrict__ seq_lens, uint32_t* status,
+    int batch, int hkv, int hg, int B, int num_pages, int max_blocks, int kw, int nchunks,
+    uint64_t* __restrict__ ws, unsigned int* __restrict__ next_item) {
+  constexpr int SC = kDecChunk / KPL;         // candidates per step = lanes per group
+  constexpr int NCW = kPass1Threads / 32;     // consumer warps
+  constexpr int NW = NCW + 1;
+  constexpr int kNoCand = -0x7fffffff - 1;
+  static_assert(SC >= 1 && SC <= 32, "a group's lanes stay inside one warp");
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  __shared__ __align__(8) uint64_t full[NST];
+  __shared__ __align__(8) uint64_t empty[NST];
+  __shared__ int s_item[NST][3];  // (b, c, gs) of the step held by each stage
+  __shared__ uint32_t s_valid[NST];  // bit k: candidate k of the step was copied
+  __shared__ int wsum[NW];
+  const int hsplit = hkv / hg;                 // items per (sequence, chunk)
+  const uint32_t page_bytes = (uint32_t)hg * D * 4;  // the item's groups of one page
+  const int pstride = (int)page_bytes + 16;   // padded: conflict-free float4 reads
+  const int stage_bytes = pass1_stage_bytes(hg, D);
+  int* pre = reinterpret_cast<int*>(smem_raw + (size_t)NST * stage_bytes);  // [batch + 1]
+  int* ncs = pre + batch + 1;                                                // [batch]
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+  if (tid == 0) {
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], NCW);
+    }
+    mbar_fence_init();
+  }
+  pdl_wait();
+  // candidates and chunk counts per sequence -> prefix sums pre[b]
+  int carry = 0;
+  for (int base = 0; base < batch; base += NW * 32) {
+    const int b = base + tid;
+    int n = 0;
+    if (b < batch) {
+      const int L = seq_lens[b];
+      int nc = 0;
+      if (L < 1 || L > max_blocks * B) {
+        if (blockIdx.x == 0) report(status, MSA_DEV_BAD_LENGTH);
+      } else {
+        nc = (L - 1) / B;
+        n = (nc + kDecChunk - 1) / kDecChunk * hsplit;
+      }
+      ncs[b] = nc;
+    }
+    int v = n;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, v, o);
+      if (lane >= o) v += t;
+    }
+    if (lane == 31) wsum[warp] = v;
+    __syncthreads();
+    int before = 0, all = 0;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) {
+      before += w < warp ? wsum[w] : 0;
+      all += wsum[w];
+    }
+    if (b < batch) pre[b + 1] = carry + before + v;
+    carry += all;
+    __syncthreads();
+  }
+  if (tid == 0) pre[0] = 0;
+  __syncthreads();
+  const int total_items = pre[batch];
+
+  if (warp == NCW) {
+    // ------------------------------ producer ------------------------------
+    // items are claimed from a shared counter when their first step is fetched
+    auto claim = [&]() {
+      unsigned int v = 0;
+      if (lane == 0) v = atomicAdd(next_item, 1u);
+      v = __shfl_sync(0xffffffffu, v, 0);
+      return v < (unsigned int)total_items ? (int)v : -1;
+    };
+    int cur_b = 0, cur_c = 0, cur_gs = 0;
+    // locate item `it` (sets cur_*); returns this lane's page entry for step `sub`
+    auto fetch = [&](int it, int sub) {
+      int lo = 0, hi = batch;  // pre[lo] <= it < pre[hi]
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (pre[mid] <= it) lo = mid; else hi = mid;
+      }
+      cur_b = lo;
+      const int r = it - pre[lo];
+      cur_c = r / hsplit;
+      cur_gs = r - cur_c * hsplit;
+      const int j = cur_c * kDecChunk + sub * SC + lane;
+      return (lane < SC && j < ncs[lo]) ? page_table[(size_t)lo * max_blocks + j] : kNoCand;
+    };
+    int it = claim(), sub = 0;
+    int pg = it >= 0 ? fetch(it, 0) : kNoCand;
+    int n = 0;
+    for (;; ++n) {
+      const int s = n % NST;
+      if (n >= NST &&
+          !__all_sync(0xffffffffu, mbar_wait(&empty[s], (uint32_t)((n / NST) - 1) & 1u))) {
+        if (lane == 0) report(status, MSA_DEV_TIMEOUT);
+        break;
+      }
+      if (it < 0) {  // no items left: an empty stage tells the consumers to stop
+        if (lane == 0) {
+          s_item[s][0] = -1;
+          mbar_expect_tx(&full[s], 0u);
+        }
+        ++n;
+        break;
+      }
+      bool valid = false;
+      if (pg != kNoCand) {
+        if (pg < 0 || pg >= num_pages) report(status, MSA_DEV_BAD_PAGE);
+        else valid = true;
+      }
+      const uint32_t vb = __ballot_sync(0xffffffffu, valid);
+      unsigned char* st = smem_raw + (size_t)s * stage_bytes;
+      if (lane == 0) {
+        s_valid[s] = vb;
+        s_item[s][0] = cur_b;
+        s_item[s][1] = cur_c;
+        s_item[s][2] = cur_gs;
+        mbar_expect_tx(&full[s], (uint32_t)(__popc(vb) + 1) * page_bytes);
+      }
+      __syncwarp();
+      if (valid)
+        bulk_load_1d(st + (size_t)lane * pstride,
+                     centroids + ((size_t)pg * hkv + (size_t)cur_gs * hg) * D, page_bytes, &full[s]);
+      if (lane == 0)
+        bulk_load_1d(st + (size_t)SC * pstride,
+                     qbar_all + ((size_t)cur_b * hkv + (size_t)cur_gs * hg) * D, page_bytes,
+                     &full[s]);
+      if (++sub == KPL) {
+        sub = 0;
+        it = claim();
+      }
+      pg = it >= 0 ? fetch(it, sub) : kNoCand;
+    }
+    // every copy issued has landed before the CTA may end
+    for (int m = n - NST < 0 ? 0 : n - NST; m < n; ++m)
+      (void)mbar_wait(&full[m % NST], (uint32_t)(m / NST) & 1u);
+    return;
+  }
+
+  // ------------------------------- consumers -------------------------------
+  const int my_g = tid / SC, my_k = tid - (tid / SC) * SC;
+  const bool active = my_g < hg;
+  int n = 0;
+#pragma unroll 1
+  for (;;) {
+    uint64_t keys[KPL];
+    int b = 0, c = 0, gs = 0;
+    bool done = false;
+#pragma unroll
+    for (int sub = 0; sub < KPL; ++sub, ++n) {
+      const int s = n % NST;
+      if (!__all_sync(0xffffffffu, mbar_wait(&full[s], (uint32_t)(n / NST) & 1u))) {
+        if (lane == 0) report(status, MSA_DEV_TIMEOUT);
+        return;
+      }
+      b = s_item[s][0];
+      if (b < 0) {  // the producer ran out of items (only at an item boundary)
+        done = true;
+        break;
+      }
+      c = s_item[s][1];
+      gs = s_item[s][2];
+      uint64_t key = 0ull;
+      if (active && ((s_valid[s] >> my_k) & 1u)) {
+        const unsigned char* st = smem_raw + (size_t)s * stage_bytes;
+        const float4* cr = reinterpret_cast<const float4*>(st + (size_t)my_k * pstride +
+                                                           (size_t)my_g * D * 4);
+        const float4* qb = reinterpret_cast<const float4*>(st + (size_t)SC * pstride +
+                                                           (size_t)my_g * D * 4);
+        float acc = 0.f;
+#pragma unroll
+        for (int x = 0; x < D / 4; ++x) {
+          const float4 cv = cr[x];
+          const float4 qv = qb[x];
+          acc = __fmaf_rn(qv.x, cv.x, acc);
+          acc = __fmaf_rn(qv.y, cv.y, acc);
+          acc = __fmaf_rn(qv.z, cv.z, acc);
+          acc = __fmaf_rn(qv.w, cv.w, acc);
+        }
+        key = sel_key(acc, c * kDecChunk + sub * SC + my_k);
+      }
+      keys[sub] = key;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+    }
+    if (done) break;
+    // bitonic sort (descending) of the group's 64 keys: element e = my_k * KPL + r
+#pragma unroll
+    for (int size = 2; size <= kDecChunk; size <<= 1) {
+#pragma unroll
+      for (int stride = size >> 1; stride > 0; stride >>= 1) {
+        if (stride >= KPL) {
+#pragma unroll
+          for (int r = 0; r < KPL; ++r) {
+            const int e = my_k * KPL + r;
+            const uint64_t o = shfl_xor_u64(keys[r], stride / KPL);
+            const bool take_max = ((e & stride) == 0) == ((e & size) == 0);
+            keys[r] = take_max ? (keys[r] > o ? keys[r] : o) : (keys[r] < o ? keys[r] : o);
+          }
+        } else {
+#pragma unroll
+          for (int r = 0; r < KPL; ++r) {
+            if ((r & stride) == 0) {
+              const int e = my_k * KPL + r;
+              const uint64_t x0 = keys[r], x1 = keys[r + stride];
+              const bool desc = (e & size) == 0;
+              const bool swap = desc ? (x0 < x1) : (x0 > x1);
+              keys[r] = swap ? x1 : x0;
+              keys[r + stride] = swap ? x0 : x1;
+            }
+          }
         }
       }
     }
-  }
-  __syncthreads();
-}
-
-template <typename T, int D>
-__global__ void __launch_bounds__(kDecChunk) select_decode_pass1(
-    const T* __restrict__ q, const float* __restrict__ centroids,
-    const int32_t* __restrict__ page_table, const int32_t* __restrict__ seq_lens, uint32_t* status,
-    int hq, int hkv, int B, int num_pages, int max_blocks, int kw, int nchunks,
-    uint64_t* __restrict__ ws) {
-  constexpr int CP = D + 4;
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  float* cent = reinterpret_cast<float*>(smem_raw);  // [kDecChunk][CP]
-  __shared__ float qbar[D];
-  __shared__ uint64_t keys[kDecChunk];
-  __shared__ int s_page[kDecChunk];
-  const int c = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
-  const int G = hq / hkv;
-  const int L = seq_lens[b];
-  uint64_t* out = ws + (((size_t)b * hkv + g) * nchunks + c) * kw;
-  if (L < 1 || L > max_blocks * B) {
-    if (c == 0 && g == 0 && threadIdx.x == 0) report(status, MSA_DEV_BAD_LENGTH);
-    for (int s = threadIdx.x; s < kw; s += blockDim.x) out[s] = 0ull;
-    return;
-  }
-  const int ncand = (L - 1) / B;
-  const int j0 = c * kDecChunk;
-  const int nc = max(0, min(kDecChunk, ncand - j0));
-  if (nc == 0) {
-    for (int s = threadIdx.x; s < kw; s += blockDim.x) out[s] = 0ull;
-    return;
-  }
-  const int tid = threadIdx.x;
-  {
-    constexpr int VEC = 16 / sizeof(T);
-    for (int i = tid * VEC; i < D; i += blockDim.x * VEC)
-      load_qbar_vec<T>(q + (size_t)b * hq * D, G, g, D, i, &qbar[i]);
-  }
-  {
-    int pg = -1;
-    if (tid < nc) {
-      pg = page_table[(size_t)b * max_blocks + j0 + tid];
-      if (pg < 0 || pg >= num_pages) {
-        report(status, MSA_DEV_BAD_PAGE);
-        pg = -1;
+    if (active) {
+      uint64_t* out = ws + (((size_t)b * hkv + gs * hg + my_g) * nchunks + c) * kw;
+#pragma unroll
+      for (int r = 0; r < KPL; ++r) {
+        const int e = my_k * KPL + r;
+        if (e < kw) out[e] = keys[r];
       }
     }
-    s_page[tid] = pg;
   }
+  pdl_release();
+}
+
+__device__ __forceinline__ uint64_t shfl_u64(uint64_t v, int src) {
+  const uint32_t lo = __shfl_sync(0xffffffffu, (uint32_t)v, src);
+  const uint32_t hi = __shfl_sync(0xffffffffu, (uint32_t)(v >> 32), src);
+  return ((uint64_t)hi << 32) | lo;
+}
+
+// Top 32 of two descending lists held one key per lane (lane l = rank l):
+// the elementwise max of one list and the other reversed is bitonic and holds
+// the top 32 of both; five half-cleaner steps sort it, descending.
+__device__ __forceinline__ uint64_t warp_merge_top32(uint64_t a, uint64_t b, int lane) {
+  const uint64_t r = shfl_u64(b, 31 - lane);
+  uint64_t x = a > r ? a : r;
+#pragma unroll
+  for (int st = 16; st > 0; st >>= 1) {
+    const uint64_t o = shfl_xor_u64(x, st);
+    x = ((lane & st) == 0) ? (x > o ? x : o) : (x < o ? x : o);
+  }
+  return x;
+}
+
+// Pass 2 for kw <= 32: a CTA of four warps per (sequence, group). A chunk list
+// is held one key per lane (one coalesced load); each warp merges eight lists
+// at a time as a balanced tree into its running top 32, warp 0 merges the four
+// warps' lists, lane l then holds rank l, and a 32-lane bitonic sort on the
+// block index gives the ascending output.
+__global__ void __launch_bounds__(128) select_decode_merge(
+    const uint64_t* __restrict__ ws, const int32_t* __restrict__ seq_lens, int hkv, int B,
+    int max_blocks, int kw, int nchunks, int top_k, int32_t* __restrict__ idx,
+    float* __restrict__ score) {
+  __shared__ uint64_t part[4][32];
+  pdl_wait();
+  const int g = blockIdx.x, b = blockIdx.y;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int L = seq_lens[b];
+  const size_t outo = ((size_t)b * hkv + g) * top_k;
+  if (L < 1 || L > max_blocks * B) return;  // reported by pass 1
+  const int own = (L - 1) / B;
+  const int keep = min(top_k - 1, own);
+  const int nch = (own + kDecChunk - 1) / kDecChunk;
+  const uint64_t* src = ws + ((size_t)b * hkv + g) * nchunks * kw;
+  uint64_t acc = 0ull;
+  for (int c0 = warp * 8; c0 < nch; c0 += 32) {
+    uint64_t l[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int c = c0 + u;
+      l[u] = (c < nch && lane < kw) ? src[(size_t)c * kw + lane] : 0ull;
+    }
+    l[0] = warp_merge_top32(l[0], l[1], lane);
+    l[2] = warp_merge_top32(l[2], l[3], lane);
+    l[4] = warp_merge_top32(l[4], l[5], lane);
+    l[6] = warp_merge_top32(l[6], l[7], lane);
+    l[0] = warp_merge_top32(l[0], l[2], lane);
+    l[4] = warp_merge_top32(l[4], l[6], lane);
+    l[0] = warp_merge_top32(l[0], l[4], lane);
+    acc = warp_merge_top32(acc, l[0], lane);
+  }
+  part[warp][lane] = acc;
   __syncthreads();
-  // stage the chunk's centroids: 16-byte async copies, one candidate row per 32 threads
-  for (int e = tid; e < nc * (D / 4); e += blockDim.x) {
-    const int jj = e / (D / 4), i4 = (e % (D / 4)) * 4;
-    float* dst = &cent[jj * CP + i4];
-    if (s_page[jj] >= 0) {
-      const float* src = centroids + ((size_t)s_page[jj] * hkv + g) * D + i4;
-      const uint32_t saddr = (uint32_t)__cvta_generic_to_shared(dst);
-      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(saddr), "l"(src));
+  if (warp != 0) return;
+  uint64_t m0 = warp_merge_top32(part[0][lane], part[1][lane], lane);
+  const uint64_t m1 = warp_merge_top32(part[2][lane], part[3][lane], lane);
+  const uint64_t mine = warp_merge_top32(m0, m1, lane);
+  const bool real = lane < keep && mine != 0ull;
+  const int cnt = __popc(__ballot_sync(0xffffffffu, real));  // fewer if pages were bad
+  int blk = real ? key_block(mine) : 0x7fffffff;
+  float sc = key_score(mine);
+#pragma unroll
+  for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      const int ob = __shfl_xor_sync(0xffffffffu, blk, stride);
+      const float os = __shfl_xor_sync(0xffffffffu, sc, stride);
+      const bool take_min = ((lane & stride) == 0) == ((lane & size) == 0);
+      if (take_min ? (ob < blk) : (ob > blk)) {
+        blk = ob;
+        sc = os;
+      }
     }
   }
-  asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;\n" ::: "memory");
-  __syncthreads();
-  uint64_t key = 0ull;
-  if (tid < nc && s_page[tid] >= 0) {
-    const float* cr = cent + tid * CP;
-    float s = 0.f;
-#pragma unroll 8
-    for (int i = 0; i < D; i += 4) {
-      const float4 cv = *reinterpret_cast<const float4*>(cr + i);
-      s = __fmaf_rn(qbar[i], cv.x, s);
-      s = __fmaf_rn(qbar[i + 1], cv.y, s);
-      s = __fmaf_rn(qbar[i + 2], cv.z, s);
-      s = __fmaf_rn(qbar[i + 3], cv.w, s);
-    }
-    key = sel_key(s, j0 + tid);
+  if (lane < cnt) {
+    idx[outo + lane] = blk;
+    if (score) score[outo + lane] = sc;
   }
-  keys[tid] = key;
-  bitonic_desc(keys, kDecChunk);
-  for (int s = tid; s < kw; s += blockDim.x) out[s] = keys[s];
+  if (lane == 0) {
+    idx[outo + cnt] = own;
+    if (score) score[outo + cnt] = __int_as_float(0x7f800000);
+  }
+  for (int s = cnt + 1 + lane; s < top_k; s += 32) {
+    idx[outo + s] = -1;
+    if (score) score[outo + s] = __int_as_float(0xff800000);
+  }
+  pdl_release();
 }
 
 // Pass 2: one warp per (sequence, group) merges the chunk lists, each already
 // sorted by pass 1, with a tournament: every round the lanes offer the heads
-// of their chunks, the warp maximum is taken and its chunk advances.
+// of their chunks, the warp maximum is taken (high then low 32 bits, keys are
+// unique) and its chunk advances.
 __global__ void __launch_bounds__(32) select_decode_pass2(
     const uint64_t* __restrict__ ws, const int32_t* __restrict__ seq_lens, int hkv, int B,
     int max_blocks, int kw, int nchunks, int top_k, int32_t* __restrict__ idx,
     float* __restrict__ score) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
+  extern __shared__ __align__(128) unsigned char smem_raw[];
   uint64_t* lists = reinterpret_cast<uint64_t*>(smem_raw);  // [nch][kw]
   __shared__ uint64_t chosen[256];
+  pdl_wait();
   const int g = blockIdx.x, b = blockIdx.y, lane = threadIdx.x;
   const int L = seq_lens[b];
   const size_t outo = ((size_t)b * hkv + g) * top_k;
@@ -389,15 +691,15 @@ __global__ void __launch_bounds__(32) select_decode_pass2(
   const int nch = (ncand + kDecChunk - 1) / kDecChunk;
   const uint64_t* src = ws + ((size_t)b * hkv + g) * nchunks * kw;
   const int total = nch * kw;
-  for (int i0 = 0; i0 < total; i0 += 8 * 32) {  // eight independent loads per lane in flight
-    uint64_t v[8];
+  for (int i0 = 0; i0 < total; i0 += 32 * 32) {  // up to 32 loads per lane in flight
+    uint64_t v[32];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
+    for (int u = 0; u < 32; ++u) {
       const int i = i0 + u * 32 + lane;
       v[u] = i < total ? src[i] : 0ull;
     }
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
+    for (int u = 0; u < 32; ++u) {
       const int i = i0 + u * 32 + lane;
       if (i < total) lists[i] = v[u];
     }
@@ -412,18 +714,16 @@ __global__ void __launch_bounds__(32) select_decode_pass2(
     head[s] = (c < nch) ? lists[(size_t)c * kw] : 0ull;
   }
   int cnt = 0;
+  const int lane_chunks = (nch + 31) / 32;
   for (; cnt < keep; ++cnt) {
-    uint64_t best = 0ull;
+    uint64_t best = head[0];
 #pragma unroll
-    for (int s = 0; s < kMaxChunksPerLane; ++s) best = head[s] > best ? head[s] : best;
-    uint64_t wb = best;
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) {
-      const uint32_t lo = __shfl_xor_sync(0xffffffffu, (uint32_t)wb, o);
-      const uint32_t hi = __shfl_xor_sync(0xffffffffu, (uint32_t)(wb >> 32), o);
-      const uint64_t other = ((uint64_t)hi << 32) | lo;
-      wb = other > wb ? other : wb;
-    }
+    for (int s = 1; s < kMaxChunksPerLane; ++s)
+      if (s < lane_chunks) best = head[s] > best ? head[s] : best;
+    const uint32_t bhi = (uint32_t)(best >> 32), blo = (uint32_t)best;
+    const uint32_t whi = __reduce_max_sync(0xffffffffu, bhi);
+    const uint32_t wlo = __reduce_max_sync(0xffffffffu, bhi == whi ? blo : 0u);
+    const uint64_t wb = ((uint64_t)whi << 32) | wlo;
     if (wb == 0ull) break;  // fewer real candidates than requested (bad pages)
 #pragma unroll
     for (int s = 0; s < kMaxChunksPerLane; ++s) {
@@ -454,6 +754,7 @@ __global__ void __launch_bounds__(32) select_decode_pass2(
     idx[outo + s] = -1;
     if (score) score[outo + s] = __int_as_float(0xff800000);
   }
+  pdl_release();
 }
 
 // ---------------------------------------------------------------------------
@@ -505,10 +806,31 @@ cudaError_t select_rows(const msa_paged_kv_t* kv, const void* q, const int32_t* 
 
 bool select_rows_supported(int top_k) { return top_k - 1 <= 64; }
 
+// KV groups per pass-1 item: all of them up to 8 (one page copy of 4 KB for
+// d 128), else the largest divisor of hkv up to 8 (hkv itself if that is 1)
+static int pass1_groups(int hkv) {
+  if (hkv <= 8) return hkv;
+  for (int d = 8; d > 1; --d)
+    if (hkv % d == 0) return d;
+  return hkv;
+}
+static size_t pass1_smem(const msa_paged_kv_t* kv, int nst) {
+  return (size_t)nst * pass1_stage_bytes(pass1_groups(kv->num_kv_heads), kv->head_dim) +
+         (size_t)(2 * kv->batch + 1) * 4;
+}
+constexpr size_t kSmemLimit = 227 * 1024 - 1024;  // dynamic + static, per CTA
+// three stages where they fit (steps of up to 8 candidates), else two
+static int pass1_stages(const msa_paged_kv_t* kv) {
+  const int kpl = kDecChunk / pass1_sc(pass1_groups(kv->num_kv_heads));
+  const int nst = kpl <= 8 ? 3 : 2;
+  return pass1_smem(kv, nst) <= kSmemLimit ? nst : 0;
+}
+
 // decode selection merges at most 32 * kMaxChunksPerLane chunk lists of
 // kDecChunk candidates
 bool select_decode_supported(const msa_paged_kv_t* kv) {
-  return kv->max_blocks_per_seq <= 32 * kMaxChunksPerLane * kDecChunk;
+  return kv->batch <= 65535 && kv->max_blocks_per_seq <= 32 * kMaxChunksPerLane * kDecChunk &&
+         kv->num_kv_heads <= kPass1Threads / 2 && pass1_stages(kv) > 0;
 }
 
 static int decode_nchunks(const msa_paged_kv_t* kv) {
@@ -516,34 +838,94 @@ static int decode_nchunks(const msa_paged_kv_t* kv) {
 }
 static int decode_kw(int top_k) { return top_k - 1 < kDecChunk ? (top_k - 1 < 1 ? 1 : top_k - 1) : kDecChunk; }
 
+// workspace: chunk lists [batch][hkv][nchunks][kw] u64, qbar [batch][hkv][D] f32,
+// pass 1's work counter
+static size_t decode_lists_bytes(const msa_paged_kv_t* kv, int top_k) {
+  const size_t b = (size_t)kv->batch * kv->num_kv_heads * decode_nchunks(kv) * decode_kw(top_k) * 8;
+  return (b + 255) & ~(size_t)255;
+}
+static size_t decode_qbar_bytes(const msa_paged_kv_t* kv) {
+  const size_t b = (size_t)kv->batch * kv->num_kv_heads * kv->head_dim * 4;
+  return (b + 255) & ~(size_t)255;
+}
 size_t select_decode_ws(const msa_paged_kv_t* kv, int top_k) {
-  return (size_t)kv->batch * kv->num_kv_heads * decode_nchunks(kv) * decode_kw(top_k) * 8;
+  return decode_lists_bytes(kv, top_k) + decode_qbar_bytes(kv) + 256;
+}
+
+// Resident pass-1 CTAs on the whole device, cached per (device, smem size).
+static int pass1_slots(const void* fn, size_t smem) {
+  static std::mutex mu;
+  static std::map<std::tuple<int, const void*, size_t>, int> cache;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  const auto key = std::make_tuple(dev, fn, smem);
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = cache.find(key);
+  if (it != cache.end()) return it->second;
+  int per_sm = 0, sms = 148;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, kPass1Threads + 32, smem) !=
+          cudaSuccess ||
+      per_sm < 1)
+    per_sm = 1;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int slots = per_sm * (sms > 0 ? sms : 148);
+  cache.emplace(key, slots);
+  return slots;
+}
+
+template <int D, int KPL, int NST>
+static cudaError_t launch_pass1(const msa_paged_kv_t* kv, const float* qbar, int kw, int nch,
+                                uint64_t* lists, unsigned int* counter, cudaStream_t st) {
+  const size_t smem = pass1_smem(kv, NST);
+  auto k1 = select_decode_pass1<D, KPL, NST>;
+  cudaError_t e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const int hg = pass1_groups(kv->num_kv_heads);
+  const long upper = (long)kv->batch * nch * (kv->num_kv_heads / hg);
+  const int grid = (int)std::max(1L, std::min<long>(upper, pass1_slots((const void*)k1, smem)));
+  return launch_pdl(k1, dim3(grid), dim3(kPass1Threads + 32), smem, st, (const float*)qbar,
+                    (const float*)kv->centroids, (const int32_t*)kv->page_table,
+                    (const int32_t*)kv->seq_lens, kv->status_word, kv->batch, kv->num_kv_heads, hg,
+                    kv->block_size, kv->num_pages, kv->max_blocks_per_seq, kw, nch, lists, counter);
+}
+
+template <int D>
+static cudaError_t pass1_dispatch(const msa_paged_kv_t* kv, const float* qbar, int kw, int nch,
+                                  uint64_t* lists, unsigned int* counter, cudaStream_t st) {
+  switch (kDecChunk / pass1_sc(pass1_groups(kv->num_kv_heads))) {
+    case 2: return launch_pass1<D, 2, 3>(kv, qbar, kw, nch, lists, counter, st);
+    case 4: return launch_pass1<D, 4, 3>(kv, qbar, kw, nch, lists, counter, st);
+    case 8: return launch_pass1<D, 8, 3>(kv, qbar, kw, nch, lists, counter, st);
+    case 16: return launch_pass1<D, 16, 2>(kv, qbar, kw, nch, lists, counter, st);
+    default: return launch_pass1<D, 32, 2>(kv, qbar, kw, nch, lists, counter, st);
+  }
 }
 
 template <typename T, int D>
 static cudaError_t launch_decode_sel(const msa_paged_kv_t* kv, const void* q, int top_k,
                                      int32_t* idx, float* score, void* ws, cudaStream_t st) {
   const int nch = decode_nchunks(kv), kw = decode_kw(top_k);
-  const size_t smem = (size_t)kDecChunk * (D + 4) * 4;
-  auto k1 = select_decode_pass1<T, D>;
-  cudaError_t e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  uint64_t* lists = (uint64_t*)ws;
+  float* qbar = (float*)((char*)ws + decode_lists_bytes(kv, top_k));
+  unsigned int* counter = (unsigned int*)((char*)qbar + decode_qbar_bytes(kv));
+  cudaError_t e = launch_pdl(select_decode_qbar<T, D>, dim3(kv->num_kv_heads, kv->batch), dim3(D),
+                             0, st, (const T*)q, kv->num_q_heads, kv->num_kv_heads, qbar, counter);
   if (e != cudaSuccess) return e;
-  dim3 g1(nch, kv->num_kv_heads, kv->batch);
-  k1<<<g1, kDecChunk, smem, st>>>((const T*)q, kv->centroids, kv->page_table, kv->seq_lens,
-                                   kv->status_word, kv->num_q_heads, kv->num_kv_heads,
-                                   kv->block_size, kv->num_pages, kv->max_blocks_per_seq, kw, nch,
-                                   (uint64_t*)ws);
-  e = cudaGetLastError();
+  e = pass1_dispatch<D>(kv, qbar, kw, nch, lists, counter, st);
   if (e != cudaSuccess) return e;
   dim3 g2(kv->num_kv_heads, kv->batch);
+  const int32_t* sl = kv->seq_lens;
+  const int hkv = kv->num_kv_heads, B = kv->block_size, mb = kv->max_blocks_per_seq;
+  if (kw <= 32)
+    return launch_pdl(select_decode_merge, g2, dim3(128), 0, st, (const uint64_t*)lists, sl, hkv,
+                      B, mb, kw, nch, top_k, idx, score);
   const size_t smem2 = (size_t)nch * kw * 8;
   e = cudaFuncSetAttribute(select_decode_pass2, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem2);
   if (e != cudaSuccess) return e;
-  select_decode_pass2<<<g2, 32, smem2, st>>>((const uint64_t*)ws, kv->seq_lens, kv->num_kv_heads,
-                                          kv->block_size, kv->max_blocks_per_seq, kw, nch, top_k,
-                                          idx, score);
-  return cudaGetLastError();
+  return launch_pdl(select_decode_pass2, g2, dim3(32), smem2, st, (const uint64_t*)lists,
+                    (const int32_t*)kv->seq_lens, kv->num_kv_heads, kv->block_size,
+                    kv->max_blocks_per_seq, kw, nch, top_k, idx, score);
 }
 
 cudaError_t select_decode(const msa_paged_kv_t* kv, const void* q, int top_k, int32_t* idx,
