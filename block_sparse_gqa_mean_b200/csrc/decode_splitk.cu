@@ -90,28 +90,46 @@ __global__ void __launch_bounds__(128) decode_splitk_kernel(
   const int t = L - 1;
   const bool len_ok = (L >= 1 && L <= max_blocks * B);
 
+  // this split's slots: one thread each looks up block and page, then the
+  // valid ones are compacted in slot order (per_split <= 256)
+  __shared__ int s_wcnt[4];
+  const int s0 = split * per_split;
+  const int nslots = len_ok ? max(0, min(top_k, s0 + per_split) - s0) : 0;
+  if (!len_ok && split == 0 && g == 0 && tid == 0) report(status, MSA_DEV_BAD_LENGTH);
   if (tid == 0) {
-    int n = 0;
-    if (len_ok) {
-      const int32_t* sel = block_idx + ((size_t)b * hkv + g) * top_k;
-      const int s0 = split * per_split, s1 = min(top_k, s0 + per_split);
-      for (int s = s0; s < s1; ++s) {
-        const int j = sel[s];
-        if (j < 0) continue;
-        if (j > t / B) { report(status, MSA_DEV_BAD_INDEX); continue; }
-        const int pg = page_table[(size_t)b * max_blocks + j];
-        if (pg < 0 || pg >= num_pages) { report(status, MSA_DEV_BAD_PAGE); continue; }
-        s_page[n] = pg;
-        s_blk[n] = j;
-        ++n;
-      }
-    } else if (split == 0 && g == 0) {
-      report(status, MSA_DEV_BAD_LENGTH);
-    }
-    s_n = n;
+    s_n = 0;
     s_abort = 0;
     for (int s = 0; s < NST; ++s) mbar_init(&full[s], 1);
     mbar_fence_init();
+  }
+  const int32_t* sel = block_idx + ((size_t)b * hkv + g) * top_k + s0;
+  for (int base = 0; base < nslots; base += 128) {
+    int j = -1, pg = -1;
+    bool ok = false;
+    if (base + tid < nslots) {
+      j = sel[base + tid];
+      if (j >= 0) {
+        if (j > t / B) {
+          report(status, MSA_DEV_BAD_INDEX);
+        } else {
+          pg = page_table[(size_t)b * max_blocks + j];
+          if (pg < 0 || pg >= num_pages) report(status, MSA_DEV_BAD_PAGE);
+          else ok = true;
+        }
+      }
+    }
+    const uint32_t bal = __ballot_sync(0xffffffffu, ok);
+    if (lane == 0) s_wcnt[warp] = __popc(bal);
+    __syncthreads();
+    int pos = s_n + __popc(bal & ((1u << lane) - 1u));
+    for (int w = 0; w < warp; ++w) pos += s_wcnt[w];
+    if (ok) {
+      s_page[pos] = pg;
+      s_blk[pos] = j;
+    }
+    __syncthreads();
+    if (tid == 0) s_n += s_wcnt[0] + s_wcnt[1] + s_wcnt[2] + s_wcnt[3];
+    __syncthreads();
   }
   __syncthreads();
   const int n = s_n;
