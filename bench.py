@@ -423,7 +423,7 @@ def run_decode(w, steps, warmup, world, flush_l2):
         raise RuntimeError(f"device status {status:#x}")
     return {"step_ms": per_step[0], "kernel_ms": k_ms, "clocks": clk.summary(),
             "e2e_ms": e2e_ms, "h2d": (hq_.numel() + hk.numel() + hv.numel()) * 2,
-            "d2h": hout.numel() * 2, "launches_per_step": 1 + 2 + 2}
+            "d2h": hout.numel() * 2, "launches_per_step": 1 + 3 + 2}
 
 
 # ---------------------------------------------------------------------------
@@ -551,20 +551,52 @@ def main():
         dist.destroy_process_group()
 
 
+def decode_call_bytes(w, step=0):
+    """Algorithmic HBM bytes of the selection call (centroid scan, q) and of the
+    attention call (K/V rows of the selected blocks, q, out)."""
+    sel = att = 0
+    for b in range(w.batch):
+        L = w.ctx[b] + step + 1
+        own = (L - 1) // w.block
+        take = min(w.top_k - 1, own)
+        keys = take * w.block + (L - own * w.block)
+        sel += w.hkv * own * w.d * 4 + w.hq * w.d * 2
+        att += w.hkv * keys * w.d * 2 * 2 + 2 * w.hq * w.d * 2
+    return sel, att
+
+
 def decode_block(w, args, world, pk):
     flush = w.name == "decode_1m_bf16"
     r = run_decode(w, args.steps, args.warmup, world, flush)
     ms = max_over_ranks(r["step_ms"], world)
     nbytes = decode_bytes(w)
+    sel_b, att_b = decode_call_bytes(w)
+    sel_ms = max_over_ranks(r["kernel_ms"][1], world)
+    att_ms = max_over_ranks(r["kernel_ms"][2], world)
+    # DRAM bytes of the two streaming kernels from their ncu summaries (paged
+    # decode workload only), None once either source has changed
+    traffic = None
+    if w.name == "paged_decode_bf16" and w.batch == 32:
+        t1 = profile_traffic("select_decode_pass1", "select.cu")
+        t2 = profile_traffic("decode_splitk_kernel", "decode_splitk.cu")
+        traffic = t1 + t2 if t1 is not None and t2 is not None else None
     return {"workload": w.name, "value": w.batch * world / (ms * 1e-3), "unit": "tokens/s",
             "ms_per_step": ms, "hbm_gbs": nbytes / (ms * 1e-3) / 1e9,
             "roofline": {"bound": "hbm", "achieved": nbytes / (ms * 1e-3) / 1e9,
                          "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": nbytes / (ms * 1e-3) / 1e9 / pk["hbm_gbs"],
-                         "traffic": None, "scope": "whole decode step (append+select+attention)",
-                         "algorithmic_bytes_per_step": nbytes},
-            "kernels_ms": {"build_block_cache": r["kernel_ms"][0], "select_topk": r["kernel_ms"][1],
-                           "sparse_attn_decode": r["kernel_ms"][2]},
+                         "traffic": traffic,
+                         "traffic_scope": "select_decode_pass1 + decode_splitk_kernel DRAM bytes",
+                         "peak_source": f"{pk['source']} HBM copy",
+                         "scope": "whole decode step (append+select+attention)",
+                         "algorithmic_bytes_per_step": nbytes,
+                         "calls": {
+                             "select_topk": {"bytes": sel_b, "ms": sel_ms,
+                                             "achieved_gbs": sel_b / (sel_ms * 1e-3) / 1e9},
+                             "sparse_attn_decode": {"bytes": att_b, "ms": att_ms,
+                                                    "achieved_gbs": att_b / (att_ms * 1e-3) / 1e9}}},
+            "kernels_ms": {"build_block_cache": r["kernel_ms"][0], "select_topk": sel_ms,
+                           "sparse_attn_decode": att_ms},
             "e2e": {"value": w.batch * world / (r["e2e_ms"] * 1e-3), "unit": "tokens/s",
                     "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
             "clocks": r["clocks"], "gpu_launches": r["launches_per_step"] * args.steps,
