@@ -594,16 +594,44 @@ __device__ __forceinline__ uint64_t warp_merge_top32(uint64_t a, uint64_t b, int
   return x;
 }
 
-// Pass 2 for kw <= 32: a CTA of four warps per (sequence, group). A chunk list
-// is held one key per lane (one coalesced load); each warp merges eight lists
-// at a time as a balanced tree into its running top 32, warp 0 merges the four
-// warps' lists, lane l then holds rank l, and a 32-lane bitonic sort on the
-// block index gives the ascending output.
+// Top 64 of two descending lists held two keys per lane (x[0] = rank l,
+// x[1] = rank l + 32): reverse + max is bitonic; the stride-32 step is inside
+// the lane, strides 16..1 are shuffles on each register.
+__device__ __forceinline__ void warp_merge_top64(uint64_t (&a)[2], const uint64_t (&b)[2],
+                                                 int lane) {
+  const uint64_t r0 = shfl_u64(b[1], 31 - lane), r1 = shfl_u64(b[0], 31 - lane);
+  uint64_t x0 = a[0] > r0 ? a[0] : r0, x1 = a[1] > r1 ? a[1] : r1;
+  const uint64_t hi = x0 > x1 ? x0 : x1, lo = x0 > x1 ? x1 : x0;
+  x0 = hi;
+  x1 = lo;
+#pragma unroll
+  for (int st = 16; st > 0; st >>= 1) {
+    const uint64_t o0 = shfl_xor_u64(x0, st), o1 = shfl_xor_u64(x1, st);
+    const bool up = (lane & st) == 0;
+    x0 = up ? (x0 > o0 ? x0 : o0) : (x0 < o0 ? x0 : o0);
+    x1 = up ? (x1 > o1 ? x1 : o1) : (x1 < o1 ? x1 : o1);
+  }
+  a[0] = x0;
+  a[1] = x1;
+}
+
+template <int NK>
+__device__ __forceinline__ void warp_merge_top(uint64_t (&a)[NK], const uint64_t (&b)[NK], int lane) {
+  if constexpr (NK == 1) a[0] = warp_merge_top32(a[0], b[0], lane);
+  else warp_merge_top64(a, b, lane);
+}
+
+// Pass 2 for kw <= 32 * NK: a CTA of four warps per (sequence, group). A chunk
+// list is held NK keys per lane (rank lane + 32 r in register r; coalesced
+// loads); each warp merges eight lists at a time as a balanced tree into its
+// running top 32·NK, warp 0 merges the four warps' lists, and a bitonic sort
+// on the block index (NK elements per lane) gives the ascending output.
+template <int NK>
 __global__ void __launch_bounds__(128) select_decode_merge(
     const uint64_t* __restrict__ ws, const int32_t* __restrict__ seq_lens, int hkv, int B,
     int max_blocks, int kw, int nchunks, int top_k, int32_t* __restrict__ idx,
     float* __restrict__ score) {
-  __shared__ uint64_t part[4][32];
+  __shared__ uint64_t part[4][32 * NK];
   pdl_wait();
   const int g = blockIdx.x, b = blockIdx.y;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -614,49 +642,90 @@ __global__ void __launch_bounds__(128) select_decode_merge(
   const int keep = min(top_k - 1, own);
   const int nch = (own + kDecChunk - 1) / kDecChunk;
   const uint64_t* src = ws + ((size_t)b * hkv + g) * nchunks * kw;
-  uint64_t acc = 0ull;
+  uint64_t acc[NK];
+#pragma unroll
+  for (int r = 0; r < NK; ++r) acc[r] = 0ull;
   for (int c0 = warp * 8; c0 < nch; c0 += 32) {
-    uint64_t l[8];
+    uint64_t l[8][NK];
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
       const int c = c0 + u;
-      l[u] = (c < nch && lane < kw) ? src[(size_t)c * kw + lane] : 0ull;
+#pragma unroll
+      for (int r = 0; r < NK; ++r) {
+        const int i = lane + 32 * r;
+        l[u][r] = (c < nch && i < kw) ? src[(size_t)c * kw + i] : 0ull;
+      }
     }
-    l[0] = warp_merge_top32(l[0], l[1], lane);
-    l[2] = warp_merge_top32(l[2], l[3], lane);
-    l[4] = warp_merge_top32(l[4], l[5], lane);
-    l[6] = warp_merge_top32(l[6], l[7], lane);
-    l[0] = warp_merge_top32(l[0], l[2], lane);
-    l[4] = warp_merge_top32(l[4], l[6], lane);
-    l[0] = warp_merge_top32(l[0], l[4], lane);
-    acc = warp_merge_top32(acc, l[0], lane);
+    warp_merge_top<NK>(l[0], l[1], lane);
+    warp_merge_top<NK>(l[2], l[3], lane);
+    warp_merge_top<NK>(l[4], l[5], lane);
+    warp_merge_top<NK>(l[6], l[7], lane);
+    warp_merge_top<NK>(l[0], l[2], lane);
+    warp_merge_top<NK>(l[4], l[6], lane);
+    warp_merge_top<NK>(l[0], l[4], lane);
+    warp_merge_top<NK>(acc, l[0], lane);
   }
-  part[warp][lane] = acc;
+#pragma unroll
+  for (int r = 0; r < NK; ++r) part[warp][lane + 32 * r] = acc[r];
   __syncthreads();
   if (warp != 0) return;
-  uint64_t m0 = warp_merge_top32(part[0][lane], part[1][lane], lane);
-  const uint64_t m1 = warp_merge_top32(part[2][lane], part[3][lane], lane);
-  const uint64_t mine = warp_merge_top32(m0, m1, lane);
-  const bool real = lane < keep && mine != 0ull;
-  const int cnt = __popc(__ballot_sync(0xffffffffu, real));  // fewer if pages were bad
-  int blk = real ? key_block(mine) : 0x7fffffff;
-  float sc = key_score(mine);
+  uint64_t m0[NK], m1[NK], m2[NK], m3[NK];
 #pragma unroll
-  for (int size = 2; size <= 32; size <<= 1) {
+  for (int r = 0; r < NK; ++r) {
+    m0[r] = part[0][lane + 32 * r];
+    m1[r] = part[1][lane + 32 * r];
+    m2[r] = part[2][lane + 32 * r];
+    m3[r] = part[3][lane + 32 * r];
+  }
+  warp_merge_top<NK>(m0, m1, lane);
+  warp_merge_top<NK>(m2, m3, lane);
+  warp_merge_top<NK>(m0, m2, lane);
+  // element e = lane + 32 r holds rank e; sort the first `keep` by block index
+  int blk[NK];
+  float sc[NK];
+  int cnt = 0;
+#pragma unroll
+  for (int r = 0; r < NK; ++r) {
+    const bool real = lane + 32 * r < keep && m0[r] != 0ull;
+    cnt += __popc(__ballot_sync(0xffffffffu, real));  // fewer if pages were bad
+    blk[r] = real ? key_block(m0[r]) : 0x7fffffff;
+    sc[r] = key_score(m0[r]);
+  }
+#pragma unroll
+  for (int size = 2; size <= 32 * NK; size <<= 1) {
 #pragma unroll
     for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      const int ob = __shfl_xor_sync(0xffffffffu, blk, stride);
-      const float os = __shfl_xor_sync(0xffffffffu, sc, stride);
-      const bool take_min = ((lane & stride) == 0) == ((lane & size) == 0);
-      if (take_min ? (ob < blk) : (ob > blk)) {
-        blk = ob;
-        sc = os;
+      if (stride == 32) {  // NK == 2, size 64: both elements in this lane, ascending
+        if (blk[0] > blk[NK - 1]) {
+          const int tb = blk[0];
+          const float ts = sc[0];
+          blk[0] = blk[NK - 1];
+          sc[0] = sc[NK - 1];
+          blk[NK - 1] = tb;
+          sc[NK - 1] = ts;
+        }
+        continue;
+      }
+#pragma unroll
+      for (int r = 0; r < NK; ++r) {
+        const int e = lane + 32 * r;
+        const int ob = __shfl_xor_sync(0xffffffffu, blk[r], stride);
+        const float os = __shfl_xor_sync(0xffffffffu, sc[r], stride);
+        const bool take_min = ((e & stride) == 0) == ((e & size) == 0);
+        if (take_min ? (ob < blk[r]) : (ob > blk[r])) {
+          blk[r] = ob;
+          sc[r] = os;
+        }
       }
     }
   }
-  if (lane < cnt) {
-    idx[outo + lane] = blk;
-    if (score) score[outo + lane] = sc;
+#pragma unroll
+  for (int r = 0; r < NK; ++r) {
+    const int e = lane + 32 * r;
+    if (e < cnt) {
+      idx[outo + e] = blk[r];
+      if (score) score[outo + e] = sc[r];
+    }
   }
   if (lane == 0) {
     idx[outo + cnt] = own;
@@ -917,8 +986,11 @@ static cudaError_t launch_decode_sel(const msa_paged_kv_t* kv, const void* q, in
   const int32_t* sl = kv->seq_lens;
   const int hkv = kv->num_kv_heads, B = kv->block_size, mb = kv->max_blocks_per_seq;
   if (kw <= 32)
-    return launch_pdl(select_decode_merge, g2, dim3(128), 0, st, (const uint64_t*)lists, sl, hkv,
-                      B, mb, kw, nch, top_k, idx, score);
+    return launch_pdl(select_decode_merge<1>, g2, dim3(128), 0, st, (const uint64_t*)lists, sl,
+                      hkv, B, mb, kw, nch, top_k, idx, score);
+  if (top_k - 1 <= 64)
+    return launch_pdl(select_decode_merge<2>, g2, dim3(128), 0, st, (const uint64_t*)lists, sl,
+                      hkv, B, mb, kw, nch, top_k, idx, score);
   const size_t smem2 = (size_t)nch * kw * 8;
   e = cudaFuncSetAttribute(select_decode_pass2, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem2);

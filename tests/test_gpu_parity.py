@@ -193,6 +193,10 @@ DECODE_CASES = [
     ("paged_g4", lambda: workloads.paged_decode_bf16(batch=4, ctx=(3000, 4095, 4096, 5000))),
     ("long_g8_b128", lambda: workloads.decode_1m_bf16(ctx=(40000,), steps=3)),
     ("varlen_g16", lambda: workloads.varlen_decode_bf16(batch=5, len_range=(1000, 20000))),
+    # k-1 > 64: the tournament merge; k = 2: one-key chunk lists
+    ("topk100", lambda: workloads.paged_decode_bf16(batch=3, ctx=(9000, 12000, 20000), top_k=100)),
+    ("topk2", lambda: workloads.paged_decode_bf16(batch=2, ctx=(5000, 700), top_k=2,
+                                                  planted=(1, 1))),
 ]
 
 
