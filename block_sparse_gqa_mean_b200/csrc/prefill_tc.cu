@@ -21,6 +21,9 @@
 // thread.
 //   TMEM columns : Q (bf16 pairs, 64) | P0 | P1 (bf16 pairs, 64 each) |
 //                  S (fp32, 128) | O (fp32, 128)
+// The row sums l are kept in the softmax threads' registers, summed over the
+// same bf16-rounded weights that P V uses (an extra row-sum MMA was measured
+// to cost the tensor pipe more than the adds cost the softmax).
 //   S = Q K^T    : M=128, N=B, K=128, A = Q (TMEM), B = K tile (K-major SW128)
 //   O += P V     : M=128, N=128, K=B, A = P (TMEM), B = V tile (MN-major SW128)
 // The softmax reads S into registers at once and releases it, so the tensor
@@ -284,14 +287,10 @@ __global__ void __launch_bounds__(192, 1) prefill_tc_kernel(
   constexpr uint32_t COL_P = 64;   // two P buffers of 64 columns (bf16 pairs)
   constexpr uint32_t COL_S = 192;  // S, 128 columns (fp32)
   constexpr uint32_t COL_O = 320;  // O, 128 columns (fp32)
-  constexpr uint32_t COL_L = 448;  // row sums of P, 16 columns (fp32; column 0 used)
-  constexpr uint32_t IDESC_L = idesc_bf16(128, 16, false);
-  constexpr int ONES = 16 * B * 2; // all-ones B operand [16][B] bf16 for the row sums
 
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  unsigned char* ones = reinterpret_cast<unsigned char*>(
+  unsigned char* stages = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-  unsigned char* stages = ones + 4096;
   __shared__ __align__(8) uint64_t kv_full[NST], kv_empty[NST];
   __shared__ __align__(8) uint64_t s_full, s_free, p_full[2], o_done[2], q_ready, fin;
   __shared__ uint32_t s_tmem;
@@ -328,9 +327,6 @@ __global__ void __launch_bounds__(192, 1) prefill_tc_kernel(
     s_abort = 0;
     mbar_fence_init();
   }
-  for (int i = tid; i < ONES / 16; i += blockDim.x)  // bf16 1.0 = 0x3f80
-    reinterpret_cast<uint4*>(ones)[i] = make_uint4(0x3f803f80u, 0x3f803f80u, 0x3f803f80u, 0x3f803f80u);
-  fence_proxy_async_smem();
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(
                      smem_u32(&s_tmem))
@@ -400,16 +396,11 @@ __global__ void __launch_bounds__(192, 1) prefill_tc_kernel(
         if (!mbar_wait(&p_full[pb], (e >> 1) & 1)) { ok = false; break; }
         tc_fence_after();
         const uint32_t vt = smem_u32(stages + (e % NST) * STAGE + TILE);
-        const uint32_t on = smem_u32(ones);
 #pragma unroll
         for (int kk = 0; kk < B / 16; ++kk) {
           const uint32_t acc = (e > 0 || kk > 0) ? 1u : 0u;
           tc_mma_ts(tmem + COL_O, tmem + COL_P + pb * 64 + kk * 8,
                     sdesc_sw128(vt + (uint32_t)kk * 2048u, (uint32_t)(TILE / 2), 1024), IDESC_O, acc);
-          // l += P * 1: the same bf16 weights, summed by the same tensor cores
-          tc_mma_ts(tmem + COL_L, tmem + COL_P + pb * 64 + kk * 8,
-                    sdesc_sw128(on + (uint32_t)(kk >> 2) * 2048u + (uint32_t)(kk & 3) * 32u, 16, 1024),
-                    IDESC_L, acc);
         }
         tc_commit(&o_done[pb]);
         tc_commit(&kv_empty[e % NST]);
@@ -457,6 +448,7 @@ __global__ void __launch_bounds__(192, 1) prefill_tc_kernel(
     // has to wait for the P*V in flight. Rows whose token did not select the
     // block use m = +inf, which turns every weight into an exact 0.
     float m_ref = -INFINITY;
+    float l_run = 0.f;  // row sum of the bf16-rounded weights P (the ones P V uses)
     const uint64_t sl2 = f2_pack(scale_log2, scale_log2);
     int2 en_next = ent[0];
     for (int e = 0; e < n_e; ++e) {
@@ -531,13 +523,7 @@ __global__ void __launch_bounds__(192, 1) prefill_tc_kernel(
           for (int xx = 0; xx < 32; ++xx) v[xx] = __float_as_uint(__uint_as_float(v[xx]) * alpha);
           tc_st32(lane_base + COL_O + c * 32, v);
         }
-        {
-          uint32_t lv[1];
-          tc_ld1(lane_base + COL_L, lv);
-          tc_wait_ld();
-          lv[0] = __float_as_uint(__uint_as_float(lv[0]) * alpha);
-          tc_st1(lane_base + COL_L, lv);
-        }
+        l_run *= alpha;
       }
       // P buffer e&1 was last read by the P*V of block e-2
       const int pb = e & 1;
@@ -551,6 +537,7 @@ __global__ void __launch_bounds__(192, 1) prefill_tc_kernel(
       // rounded weights into l, so the output is an exact convex combination)
       const float m_use = sel ? m_ref : INFINITY;
       const uint64_t neg_m = f2_pack(-m_use, -m_use);
+      uint64_t lsum2 = 0ull;  // two fp32 partial sums
 #pragma unroll
       for (int cc = 0; cc < B / 64; ++cc) {
         uint32_t pv[32];
@@ -558,7 +545,7 @@ __global__ void __launch_bounds__(192, 1) prefill_tc_kernel(
 #pragma unroll
           for (int xx = 0; xx < 32; ++xx) {
             const uint64_t arg = f2_fma(f2_pack(s[64 * cc + 2 * xx], s[64 * cc + 2 * xx + 1]), sl2, neg_m);
-            if (xx & 1) {  // every other pair on the FMA pipe, the rest on MUFU
+            if ((xx & 3) == 0) {  // one pair in four on the FMA pipe, the rest on MUFU
               float p0, p1;
               exp2_poly_pair(arg, p0, p1);
               pv[xx] = pack_bf16(p0, p1);
@@ -566,6 +553,8 @@ __global__ void __launch_bounds__(192, 1) prefill_tc_kernel(
               pv[xx] = pack_bf16(fast_exp2(__uint_as_float((uint32_t)arg)),
                                  fast_exp2(__uint_as_float((uint32_t)(arg >> 32))));
             }
+            // the rounded pair, widened back to fp32, into the row sum
+            lsum2 = f2_add(lsum2, ((uint64_t)(pv[xx] & 0xffff0000u) << 32) | (uint64_t)(pv[xx] << 16));
           }
         } else {
 #pragma unroll
@@ -576,18 +565,13 @@ __global__ void __launch_bounds__(192, 1) prefill_tc_kernel(
       tc_wait_st();
       tc_fence_before();
       mbar_arrive(&p_full[pb]);
+      l_run += __uint_as_float((uint32_t)lsum2) + __uint_as_float((uint32_t)(lsum2 >> 32));
     }
     // epilogue: O / l -> bf16 once the last P*V has completed
     const bool go = !__any_sync(0xffffffffu, s_abort != 0);
     if (go && __all_sync(0xffffffffu, mbar_wait(&o_done[(n_e - 1) & 1], ((n_e - 1) >> 1) & 1))) {
       tc_fence_after();
-      float l;
-      {
-        uint32_t lv[1];
-        tc_ld1(lane_base + COL_L, lv);
-        tc_wait_ld();
-        l = __uint_as_float(lv[0]);
-      }
+      const float l = l_run;
       const float inv = (l > 0.f) ? 1.f / l : 0.f;
       uint4* dst = reinterpret_cast<uint4*>(
           out + ((size_t)(row0 + r_lo + ti) * hq + (size_t)g * G + h) * kD);
@@ -654,7 +638,7 @@ static cudaError_t launch_tc(const msa_paged_kv_t* kv, const CUtensorMap& tk, co
                              const int2* entries, const int* counts, float sl2, void* out,
                              float* lse, cudaStream_t st) {
   constexpr int NST = (B == 128) ? 3 : 4;
-  const size_t smem = 4096 + (size_t)NST * 2 * B * kD * 2 + 1024;
+  const size_t smem = (size_t)NST * 2 * B * kD * 2 + 1024;
   auto kern = prefill_tc_kernel<B, G>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
