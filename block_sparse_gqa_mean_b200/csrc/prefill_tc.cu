@@ -525,14 +525,10 @@ __global__ void __launch_bounds__(192, 1) prefill_tc_kernel(
         }
         l_run *= alpha;
       }
-      // P buffer e&1 was last read by the P*V of block e-2
+      // P buffer e&1 was last read by the P*V of block e-2. That P*V was issued
+      // by the MMA thread before S_e, and the commit that signalled s_full for
+      // S_e tracks every earlier MMA of that thread, so it has completed.
       const int pb = e & 1;
-      if (e >= 2 && !__all_sync(0xffffffffu, mbar_wait(&o_done[pb], ((e >> 1) - 1) & 1))) {
-        report(status, MSA_DEV_TIMEOUT);
-        s_abort = 1;
-        break;
-      }
-      tc_fence_after();
       // P = exp2(s*c - m_ref) rounded to bf16 (the tensor cores sum the same
       // rounded weights into l, so the output is an exact convex combination)
       const float m_use = sel ? m_ref : INFINITY;
