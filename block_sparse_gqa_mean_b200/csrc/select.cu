@@ -623,10 +623,11 @@ __device__ __forceinline__ void warp_merge_top(uint64_t (&a)[NK], const uint64_t
 
 // Pass 2 for kw <= 32 * NK: a CTA of four warps per (sequence, group). A chunk
 // list is held NK keys per lane (rank lane + 32 r in register r; coalesced
-// loads); each warp merges eight lists at a time as a balanced tree into its
-// running top 32·NK, warp 0 merges the four warps' lists, and a bitonic sort
-// on the block index (NK elements per lane) gives the ascending output.
-template <int NK>
+// loads); each warp loads LG lists at once and merges them as a balanced tree
+// into its running top 32·NK, warp 0 merges the four warps' lists, and a
+// bitonic sort on the block index (NK elements per lane) gives the ascending
+// output.
+template <int NK, int LG>
 __global__ void __launch_bounds__(128) select_decode_merge(
     const uint64_t* __restrict__ ws, const int32_t* __restrict__ seq_lens, int hkv, int B,
     int max_blocks, int kw, int nchunks, int top_k, int32_t* __restrict__ idx,
@@ -645,10 +646,10 @@ __global__ void __launch_bounds__(128) select_decode_merge(
   uint64_t acc[NK];
 #pragma unroll
   for (int r = 0; r < NK; ++r) acc[r] = 0ull;
-  for (int c0 = warp * 8; c0 < nch; c0 += 32) {
-    uint64_t l[8][NK];
+  for (int c0 = warp * LG; c0 < nch; c0 += 4 * LG) {
+    uint64_t l[LG][NK];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
+    for (int u = 0; u < LG; ++u) {
       const int c = c0 + u;
 #pragma unroll
       for (int r = 0; r < NK; ++r) {
@@ -656,13 +657,11 @@ __global__ void __launch_bounds__(128) select_decode_merge(
         l[u][r] = (c < nch && i < kw) ? src[(size_t)c * kw + i] : 0ull;
       }
     }
-    warp_merge_top<NK>(l[0], l[1], lane);
-    warp_merge_top<NK>(l[2], l[3], lane);
-    warp_merge_top<NK>(l[4], l[5], lane);
-    warp_merge_top<NK>(l[6], l[7], lane);
-    warp_merge_top<NK>(l[0], l[2], lane);
-    warp_merge_top<NK>(l[4], l[6], lane);
-    warp_merge_top<NK>(l[0], l[4], lane);
+#pragma unroll
+    for (int w = 1; w < LG; w <<= 1) {
+#pragma unroll
+      for (int u = 0; u < LG; u += 2 * w) warp_merge_top<NK>(l[u], l[u + w], lane);
+    }
     warp_merge_top<NK>(acc, l[0], lane);
   }
 #pragma unroll
@@ -985,12 +984,19 @@ static cudaError_t launch_decode_sel(const msa_paged_kv_t* kv, const void* q, in
   dim3 g2(kv->num_kv_heads, kv->batch);
   const int32_t* sl = kv->seq_lens;
   const int hkv = kv->num_kv_heads, B = kv->block_size, mb = kv->max_blocks_per_seq;
-  if (kw <= 32)
-    return launch_pdl(select_decode_merge<1>, g2, dim3(128), 0, st, (const uint64_t*)lists, sl,
-                      hkv, B, mb, kw, nch, top_k, idx, score);
-  if (top_k - 1 <= 64)
-    return launch_pdl(select_decode_merge<2>, g2, dim3(128), 0, st, (const uint64_t*)lists, sl,
-                      hkv, B, mb, kw, nch, top_k, idx, score);
+  // lists per warp and round: enough that the four warps take them in one round
+  const int lg = nch <= 32 ? 8 : (nch <= 64 ? 16 : 32);
+  if (kw <= 32) {
+    auto k = lg == 8 ? select_decode_merge<1, 8>
+                     : (lg == 16 ? select_decode_merge<1, 16> : select_decode_merge<1, 32>);
+    return launch_pdl(k, g2, dim3(128), 0, st, (const uint64_t*)lists, sl, hkv, B, mb, kw, nch,
+                      top_k, idx, score);
+  }
+  if (top_k - 1 <= 64) {
+    auto k = lg == 8 ? select_decode_merge<2, 8> : select_decode_merge<2, 16>;
+    return launch_pdl(k, g2, dim3(128), 0, st, (const uint64_t*)lists, sl, hkv, B, mb, kw, nch,
+                      top_k, idx, score);
+  }
   const size_t smem2 = (size_t)nch * kw * 8;
   e = cudaFuncSetAttribute(select_decode_pass2, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem2);
