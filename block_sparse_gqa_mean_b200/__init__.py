@@ -33,7 +33,8 @@ MSA_OP_SELECT, MSA_OP_PREFILL, MSA_OP_DECODE = 0, 1, 2
 MSA_DEV_BAD_PAGE, MSA_DEV_BAD_LENGTH, MSA_DEV_BAD_INDEX, MSA_DEV_TIMEOUT = 1, 2, 4, 8
 
 EXPORTS = ("msa_build_block_cache", "msa_select_topk", "msa_sparse_attn_prefill",
-           "msa_sparse_attn_decode", "msa_sparse_attn_decode_noalloc", "msa_workspace_size",
+           "msa_sparse_attn_decode", "msa_sparse_attn_prefill_gated",
+           "msa_sparse_attn_decode_gated", "msa_sparse_attn_decode_noalloc", "msa_workspace_size",
            "msa_status_string", "msa_version")
 
 
@@ -82,13 +83,18 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                                             SZ, P]
     lib.msa_sparse_attn_decode.argtypes = [KV, P, P, I32, ctypes.c_float, P, P, P, SZ, P]
     lib.msa_sparse_attn_decode_noalloc.argtypes = [KV, P, P, I32, ctypes.c_float, P, P, P]
+    lib.msa_sparse_attn_prefill_gated.argtypes = [KV, P, P, I32, I32, P, I32, ctypes.c_float, P,
+                                                  I32, P, P, P, P, SZ, P]
+    lib.msa_sparse_attn_decode_gated.argtypes = [KV, P, P, I32, ctypes.c_float, P, I32, P, P, P, P,
+                                                 SZ, P]
     lib.msa_workspace_size.argtypes = [ctypes.c_int, KV, I32, I32, I32]
     lib.msa_workspace_size.restype = SZ
     lib.msa_status_string.argtypes = [ctypes.c_int]
     lib.msa_status_string.restype = ctypes.c_char_p
     lib.msa_version.restype = I32
     for name in ("msa_build_block_cache", "msa_select_topk", "msa_sparse_attn_prefill",
-                 "msa_sparse_attn_decode", "msa_sparse_attn_decode_noalloc"):
+                 "msa_sparse_attn_decode", "msa_sparse_attn_prefill_gated",
+                 "msa_sparse_attn_decode_gated", "msa_sparse_attn_decode_noalloc"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -238,10 +244,13 @@ def sparse_attn_prefill(cache: PagedKVCache, q: torch.Tensor, block_idx: torch.T
                         cu_q: torch.Tensor, max_rows_per_seq: int,
                         softmax_scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
                         lse: Optional[torch.Tensor] = None, want_lse: bool = True,
-                        workspace: Optional[torch.Tensor] = None, stream=None):
-    """Exact attention of the query rows over their selected blocks."""
+                        workspace: Optional[torch.Tensor] = None, stream=None,
+                        gate: Optional[torch.Tensor] = None, x: Optional[torch.Tensor] = None):
+    """Exact attention of the query rows over their selected blocks. With `gate`
+    (fp32, [rows, Hq] or [rows, Hq, d]) and `x` ([rows, Hq, d]) the output is
+    gate * attention + (1 - gate) * x, fused into the kernel's epilogue."""
     lib = load_library()
-    _require_cuda(q, block_idx, cu_q, out, lse)
+    _require_cuda(q, block_idx, cu_q, out, lse, gate, x)
     rows, top_k = q.shape[0], block_idx.shape[-1]
     scale = 1.0 / math.sqrt(cache.head_dim) if softmax_scale is None else softmax_scale
     if out is None:
@@ -250,6 +259,14 @@ def sparse_attn_prefill(cache: PagedKVCache, q: torch.Tensor, block_idx: torch.T
         lse = torch.empty(rows, q.shape[1], dtype=torch.float32, device=q.device)
     ws, ws_bytes = _workspace(MSA_OP_PREFILL, cache, rows, max_rows_per_seq, top_k, workspace)
     kv = cache.struct()
+    if gate is not None:
+        per_dim = _gate_layout(gate, x, q)
+        _check(lib.msa_sparse_attn_prefill_gated(ctypes.byref(kv), _ptr(q), _ptr(cu_q), rows,
+                                                 max_rows_per_seq, _ptr(block_idx), top_k, scale,
+                                                 _ptr(gate), per_dim, _ptr(x), _ptr(out),
+                                                 _ptr(lse), _ptr(ws), ws_bytes, _stream(stream)),
+               "msa_sparse_attn_prefill_gated")
+        return out, lse
     _check(lib.msa_sparse_attn_prefill(ctypes.byref(kv), _ptr(q), _ptr(cu_q), rows,
                                        max_rows_per_seq, _ptr(block_idx), top_k, scale, _ptr(out),
                                        _ptr(lse), _ptr(ws), ws_bytes, _stream(stream)),
@@ -260,10 +277,12 @@ def sparse_attn_prefill(cache: PagedKVCache, q: torch.Tensor, block_idx: torch.T
 def sparse_attn_decode(cache: PagedKVCache, q: torch.Tensor, block_idx: torch.Tensor,
                        softmax_scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
                        lse: Optional[torch.Tensor] = None, want_lse: bool = True,
-                       workspace: Optional[torch.Tensor] = None, stream=None):
-    """Attention of one new query per sequence (at seq_lens-1) over its selected blocks."""
+                       workspace: Optional[torch.Tensor] = None, stream=None,
+                       gate: Optional[torch.Tensor] = None, x: Optional[torch.Tensor] = None):
+    """Attention of one new query per sequence (at seq_lens-1) over its selected
+    blocks; `gate` and `x` as for sparse_attn_prefill."""
     lib = load_library()
-    _require_cuda(q, block_idx, out, lse)
+    _require_cuda(q, block_idx, out, lse, gate, x)
     top_k = block_idx.shape[-1]
     scale = 1.0 / math.sqrt(cache.head_dim) if softmax_scale is None else softmax_scale
     if out is None:
@@ -272,10 +291,30 @@ def sparse_attn_decode(cache: PagedKVCache, q: torch.Tensor, block_idx: torch.Te
         lse = torch.empty(q.shape[0], q.shape[1], dtype=torch.float32, device=q.device)
     ws, ws_bytes = _workspace(MSA_OP_DECODE, cache, q.shape[0], 1, top_k, workspace)
     kv = cache.struct()
+    if gate is not None:
+        per_dim = _gate_layout(gate, x, q)
+        _check(lib.msa_sparse_attn_decode_gated(ctypes.byref(kv), _ptr(q), _ptr(block_idx), top_k,
+                                                scale, _ptr(gate), per_dim, _ptr(x), _ptr(out),
+                                                _ptr(lse), _ptr(ws), ws_bytes, _stream(stream)),
+               "msa_sparse_attn_decode_gated")
+        return out, lse
     _check(lib.msa_sparse_attn_decode(ctypes.byref(kv), _ptr(q), _ptr(block_idx), top_k, scale,
                                       _ptr(out), _ptr(lse), _ptr(ws), ws_bytes, _stream(stream)),
            "msa_sparse_attn_decode")
     return out, lse
+
+
+def _gate_layout(gate: torch.Tensor, x: Optional[torch.Tensor], q: torch.Tensor) -> int:
+    """Checks the gate and x tensors; returns 1 for a per-coordinate gate."""
+    if x is None or x.shape != q.shape or x.dtype != q.dtype or not x.is_contiguous():
+        raise ValueError("x must be a contiguous tensor shaped and typed like q")
+    if gate.dtype != torch.float32 or not gate.is_contiguous():
+        raise ValueError("gate must be a contiguous fp32 tensor")
+    if tuple(gate.shape) == tuple(q.shape):
+        return 1
+    if tuple(gate.shape) == tuple(q.shape[:2]):
+        return 0
+    raise ValueError("gate must be shaped [rows, Hq] or [rows, Hq, d]")
 
 
 def sparse_attn_decode_noalloc(cache: PagedKVCache, q: torch.Tensor, block_idx: torch.Tensor,

@@ -22,7 +22,7 @@ __global__ void __launch_bounds__(128) attn_simt_kernel(
     const T* __restrict__ v_pages, const int32_t* __restrict__ page_table,
     const int32_t* __restrict__ seq_lens, uint32_t* status, const int32_t* __restrict__ block_idx,
     int top_k, int hq, int hkv, int B, int num_pages, int max_blocks, float scale,
-    T* __restrict__ out, float* __restrict__ lse) {
+    T* __restrict__ out, float* __restrict__ lse, gate_t gate) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int G = hq / hkv;
   float* qs = reinterpret_cast<float*>(smem_raw);  // [G][D]
@@ -126,7 +126,8 @@ __global__ void __launch_bounds__(128) attn_simt_kernel(
   __syncthreads();
   for (int e = tid; e < G * D; e += blockDim.x) {
     const int h = e / D;
-    out[((size_t)row * hq + g * G) * D + e] = from_f32<T>(os[e] / l_s[h]);
+    out[((size_t)row * hq + g * G) * D + e] = from_f32<T>(
+        gate_apply<T>(gate, (size_t)row * hq + g * G + h, e - h * D, D, os[e] / l_s[h]));
   }
   if (lse && tid < G) lse[(size_t)row * hq + g * G + tid] = m_s[tid] + logf(l_s[tid]);
 }
@@ -134,7 +135,7 @@ __global__ void __launch_bounds__(128) attn_simt_kernel(
 template <typename T, int D>
 static cudaError_t launch_simt(const msa_paged_kv_t* kv, const void* q, const int32_t* cu_q,
                                int grid_rows, const int32_t* idx, int top_k, float scale,
-                               void* out, float* lse, cudaStream_t st) {
+                               void* out, float* lse, gate_t gate, cudaStream_t st) {
   const int G = kv->num_q_heads / kv->num_kv_heads, B = kv->block_size;
   const size_t smem = ((size_t)2 * G * D + (size_t)B * (D + 1) + (size_t)B * D + (size_t)G * B) * 4;
   auto kern = attn_simt_kernel<T, D>;
@@ -144,20 +145,20 @@ static cudaError_t launch_simt(const msa_paged_kv_t* kv, const void* q, const in
   kern<<<grid, 128, smem, st>>>((const T*)q, cu_q, (const T*)kv->k_pages, (const T*)kv->v_pages,
                                  kv->page_table, kv->seq_lens, kv->status_word, idx, top_k,
                                  kv->num_q_heads, kv->num_kv_heads, B, kv->num_pages,
-                                 kv->max_blocks_per_seq, scale, (T*)out, lse);
+                                 kv->max_blocks_per_seq, scale, (T*)out, lse, gate);
   return cudaGetLastError();
 }
 
 // grid_rows: max rows per sequence (prefill, cu_q != NULL) or 1 (decode, cu_q == NULL)
 cudaError_t attn_simt(const msa_paged_kv_t* kv, const void* q, const int32_t* cu_q, int grid_rows,
                       const int32_t* idx, int top_k, float scale, void* out, float* lse,
-                      cudaStream_t st) {
+                      gate_t gate, cudaStream_t st) {
   const bool bf = kv->dtype == MSA_DTYPE_BF16;
   if (kv->head_dim == 128)
-    return bf ? launch_simt<bf16, 128>(kv, q, cu_q, grid_rows, idx, top_k, scale, out, lse, st)
-              : launch_simt<float, 128>(kv, q, cu_q, grid_rows, idx, top_k, scale, out, lse, st);
-  return bf ? launch_simt<bf16, 64>(kv, q, cu_q, grid_rows, idx, top_k, scale, out, lse, st)
-            : launch_simt<float, 64>(kv, q, cu_q, grid_rows, idx, top_k, scale, out, lse, st);
+    return bf ? launch_simt<bf16, 128>(kv, q, cu_q, grid_rows, idx, top_k, scale, out, lse, gate, st)
+              : launch_simt<float, 128>(kv, q, cu_q, grid_rows, idx, top_k, scale, out, lse, gate, st);
+  return bf ? launch_simt<bf16, 64>(kv, q, cu_q, grid_rows, idx, top_k, scale, out, lse, gate, st)
+            : launch_simt<float, 64>(kv, q, cu_q, grid_rows, idx, top_k, scale, out, lse, gate, st);
 }
 
 }  // namespace msa

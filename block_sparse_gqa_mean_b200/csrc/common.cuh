@@ -93,4 +93,24 @@ __device__ __forceinline__ float key_score(uint64_t k) {
   return __uint_as_float(b);
 }
 
+// Output gate fused into the attention epilogues ("Sparse Attention for
+// Long-Context LLMs: Evolution and Practical Deployment", section 4.3, step 6
+// of the computation flow): O = g * A + (1 - g) * X with g and X from the
+// caller (the gate may be a scalar or vary with the dimension); g is one value per (row, head), or one per (row, head, coordinate)
+// when per_dim is set. g == nullptr: no gate, O = A.
+struct gate_t {
+  const float* g = nullptr;
+  const void* x = nullptr;
+  int per_dim = 0;
+};
+
+// head = row * num_q_heads + query head; c = coordinate; a = attention output
+template <typename T>
+__device__ __forceinline__ float gate_apply(const gate_t& gt, size_t head, int c, int D, float a) {
+  if (!gt.g) return a;
+  const float gv = gt.per_dim ? gt.g[head * D + c] : gt.g[head];
+  const float xv = to_f32(reinterpret_cast<const T*>(gt.x)[head * D + c]);
+  return fmaf(gv, a - xv, xv);
+}
+
 }  // namespace msa

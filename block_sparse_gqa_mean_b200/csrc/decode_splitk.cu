@@ -320,7 +320,7 @@ template <typename T>
 __global__ void __launch_bounds__(128) decode_combine_kernel(const float* __restrict__ ws_o,
                                                              const float* __restrict__ ws_lse,
                                                              int splits, T* __restrict__ out,
-                                                             float* __restrict__ lse) {
+                                                             float* __restrict__ lse, gate_t gate) {
   pdl_wait();
   const size_t bh = blockIdx.x;
   const int tid = threadIdx.x;
@@ -334,7 +334,7 @@ __global__ void __launch_bounds__(128) decode_combine_kernel(const float* __rest
       w += f;
     }
   }
-  out[bh * kD + tid] = from_f32<T>(w > 0.f ? acc / w : 0.f);
+  out[bh * kD + tid] = from_f32<T>(gate_apply<T>(gate, bh, tid, kD, w > 0.f ? acc / w : 0.f));
   if (lse && tid == 0) lse[bh] = (M + log2f(w)) * 0.6931471805599453f;
   pdl_release();
 }
@@ -364,7 +364,7 @@ static size_t decode_smem(int B) {
 }
 
 cudaError_t decode_splitk(const msa_paged_kv_t* kv, const void* q, const int32_t* idx, int top_k,
-                          float scale, void* out, float* lse, void* ws, int num_sms,
+                          float scale, void* out, float* lse, void* ws, int num_sms, gate_t gate,
                           cudaStream_t st) {
   const int B = kv->block_size;
   const int splits = decode_splits(kv, top_k, num_sms);
@@ -400,7 +400,7 @@ cudaError_t decode_splitk(const msa_paged_kv_t* kv, const void* q, const int32_t
   }
   if (e != cudaSuccess) return e;
   return launch_pdl(decode_combine_kernel<bf16>, dim3(kv->batch * kv->num_q_heads), dim3(128), 0,
-                    st, (const float*)ws_o, (const float*)ws_lse, splits, (bf16*)out, lse);
+                    st, (const float*)ws_o, (const float*)ws_lse, splits, (bf16*)out, lse, gate);
 }
 
 }  // namespace msa

@@ -19,14 +19,14 @@ size_t select_decode_ws(const msa_paged_kv_t*, int top_k);
 cudaError_t select_decode(const msa_paged_kv_t*, const void*, int, int32_t*, float*, void*,
                           cudaStream_t);
 cudaError_t attn_simt(const msa_paged_kv_t*, const void*, const int32_t*, int, const int32_t*, int,
-                      float, void*, float*, cudaStream_t);
+                      float, void*, float*, gate_t, cudaStream_t);
 size_t decode_ws(const msa_paged_kv_t*, int top_k, int num_sms);
 cudaError_t decode_splitk(const msa_paged_kv_t*, const void*, const int32_t*, int, float, void*,
-                          float*, void*, int, cudaStream_t);
+                          float*, void*, int, gate_t, cudaStream_t);
 bool prefill_tc_supported(const msa_paged_kv_t*);
 size_t prefill_ws(const msa_paged_kv_t*, int max_rows, int top_k);
 cudaError_t prefill_tc(const msa_paged_kv_t*, const void*, const int32_t*, int, const int32_t*,
-                       int, float, void*, float*, void*, cudaStream_t);
+                       int, float, void*, float*, void*, gate_t, cudaStream_t);
 
 // ---------------------------------------------------------------------------
 // tensor maps (driver entry point resolved once through the runtime)
@@ -173,11 +173,11 @@ msa_status_t msa_select_topk(const msa_paged_kv_t* kv, const void* q, const int3
   return from_cuda(select_rows(kv, q, cu_q, max_rows_per_seq, top_k, block_idx, block_score, st));
 }
 
-msa_status_t msa_sparse_attn_prefill(const msa_paged_kv_t* kv, const void* q, const int32_t* cu_q,
-                                     int32_t num_rows, int32_t max_rows_per_seq,
-                                     const int32_t* block_idx, int32_t top_k, float softmax_scale,
-                                     void* out, float* lse, void* workspace,
-                                     size_t workspace_bytes, msa_stream_t stream) {
+static msa_status_t attn_prefill(const msa_paged_kv_t* kv, const void* q, const int32_t* cu_q,
+                                 int32_t num_rows, int32_t max_rows_per_seq,
+                                 const int32_t* block_idx, int32_t top_k, float softmax_scale,
+                                 gate_t gate, void* out, float* lse, void* workspace,
+                                 size_t workspace_bytes, msa_stream_t stream) {
   msa_status_t s = check_kv(kv);
   if (s != MSA_OK) return s;
   if (top_k < 1 || top_k > 256) return MSA_ERR_UNSUPPORTED;
@@ -192,16 +192,16 @@ msa_status_t msa_sparse_attn_prefill(const msa_paged_kv_t* kv, const void* q, co
     const size_t need = prefill_ws(kv, max_rows_per_seq, top_k);
     if (workspace_bytes < need || !workspace || !aligned(workspace, 16)) return MSA_ERR_WORKSPACE;
     return from_cuda(prefill_tc(kv, q, cu_q, max_rows_per_seq, block_idx, top_k, softmax_scale, out,
-                                lse, workspace, st));
+                                lse, workspace, gate, st));
   }
   return from_cuda(attn_simt(kv, q, cu_q, max_rows_per_seq, block_idx, top_k, softmax_scale, out,
-                             lse, st));
+                             lse, gate, st));
 }
 
-msa_status_t msa_sparse_attn_decode(const msa_paged_kv_t* kv, const void* q,
-                                    const int32_t* block_idx, int32_t top_k, float softmax_scale,
-                                    void* out, float* lse, void* workspace, size_t workspace_bytes,
-                                    msa_stream_t stream) {
+static msa_status_t attn_decode(const msa_paged_kv_t* kv, const void* q, const int32_t* block_idx,
+                                int32_t top_k, float softmax_scale, gate_t gate, void* out,
+                                float* lse, void* workspace, size_t workspace_bytes,
+                                msa_stream_t stream) {
   msa_status_t s = check_kv(kv);
   if (s != MSA_OK) return s;
   if (top_k < 1 || top_k > 256) return MSA_ERR_UNSUPPORTED;
@@ -214,9 +214,62 @@ msa_status_t msa_sparse_attn_decode(const msa_paged_kv_t* kv, const void* q,
     const size_t need = decode_ws(kv, top_k, sms);
     if (workspace_bytes < need || !workspace || !aligned(workspace, 16)) return MSA_ERR_WORKSPACE;
     return from_cuda(
-        decode_splitk(kv, q, block_idx, top_k, softmax_scale, out, lse, workspace, sms, st));
+        decode_splitk(kv, q, block_idx, top_k, softmax_scale, out, lse, workspace, sms, gate, st));
   }
-  return from_cuda(attn_simt(kv, q, nullptr, 1, block_idx, top_k, softmax_scale, out, lse, st));
+  return from_cuda(
+      attn_simt(kv, q, nullptr, 1, block_idx, top_k, softmax_scale, out, lse, gate, st));
+}
+
+static bool gate_ok(const float* gate, int32_t per_dim, const void* x) {
+  return gate && x && aligned(gate, 4) && aligned(x, 16) && (per_dim == 0 || per_dim == 1);
+}
+
+msa_status_t msa_sparse_attn_prefill(const msa_paged_kv_t* kv, const void* q, const int32_t* cu_q,
+                                     int32_t num_rows, int32_t max_rows_per_seq,
+                                     const int32_t* block_idx, int32_t top_k, float softmax_scale,
+                                     void* out, float* lse, void* workspace,
+                                     size_t workspace_bytes, msa_stream_t stream) {
+  return attn_prefill(kv, q, cu_q, num_rows, max_rows_per_seq, block_idx, top_k, softmax_scale,
+                      gate_t{}, out, lse, workspace, workspace_bytes, stream);
+}
+
+msa_status_t msa_sparse_attn_prefill_gated(const msa_paged_kv_t* kv, const void* q,
+                                           const int32_t* cu_q, int32_t num_rows,
+                                           int32_t max_rows_per_seq, const int32_t* block_idx,
+                                           int32_t top_k, float softmax_scale, const float* gate,
+                                           int32_t gate_per_dim, const void* x, void* out,
+                                           float* lse, void* workspace, size_t workspace_bytes,
+                                           msa_stream_t stream) {
+  if (!gate_ok(gate, gate_per_dim, x)) return MSA_ERR_INVALID_ARG;
+  gate_t gt;
+  gt.g = gate;
+  gt.x = x;
+  gt.per_dim = gate_per_dim;
+  return attn_prefill(kv, q, cu_q, num_rows, max_rows_per_seq, block_idx, top_k, softmax_scale, gt,
+                      out, lse, workspace, workspace_bytes, stream);
+}
+
+msa_status_t msa_sparse_attn_decode(const msa_paged_kv_t* kv, const void* q,
+                                    const int32_t* block_idx, int32_t top_k, float softmax_scale,
+                                    void* out, float* lse, void* workspace, size_t workspace_bytes,
+                                    msa_stream_t stream) {
+  return attn_decode(kv, q, block_idx, top_k, softmax_scale, gate_t{}, out, lse, workspace,
+                     workspace_bytes, stream);
+}
+
+msa_status_t msa_sparse_attn_decode_gated(const msa_paged_kv_t* kv, const void* q,
+                                          const int32_t* block_idx, int32_t top_k,
+                                          float softmax_scale, const float* gate,
+                                          int32_t gate_per_dim, const void* x, void* out,
+                                          float* lse, void* workspace, size_t workspace_bytes,
+                                          msa_stream_t stream) {
+  if (!gate_ok(gate, gate_per_dim, x)) return MSA_ERR_INVALID_ARG;
+  gate_t gt;
+  gt.g = gate;
+  gt.x = x;
+  gt.per_dim = gate_per_dim;
+  return attn_decode(kv, q, block_idx, top_k, softmax_scale, gt, out, lse, workspace,
+                     workspace_bytes, stream);
 }
 
 }  // extern "C"

@@ -275,7 +275,7 @@ __global__ void __launch_bounds__(192, 1) prefill_tc_kernel(
     const int32_t* __restrict__ page_table, const int32_t* __restrict__ seq_lens, uint32_t* status,
     int hq, int hkv, int num_pages, int max_blocks, int units_per_seq, int ecap,
     const int2* __restrict__ entries, const int* __restrict__ counts, float scale_log2,
-    bf16* __restrict__ out, float* __restrict__ lse) {
+    bf16* __restrict__ out, float* __restrict__ lse, gate_t gate) {
   constexpr int TM = 128 / G;              // tokens per query tile (128 rows)
   constexpr int NST = (B == 128) ? 3 : 4;  // K+V stages
   constexpr int TILE = B * kD * 2;         // bytes of a K (or V) tile
@@ -569,14 +569,28 @@ __global__ void __launch_bounds__(192, 1) prefill_tc_kernel(
       tc_fence_after();
       const float l = l_run;
       const float inv = (l > 0.f) ? 1.f / l : 0.f;
-      uint4* dst = reinterpret_cast<uint4*>(
-          out + ((size_t)(row0 + r_lo + ti) * hq + (size_t)g * G + h) * kD);
+      const size_t head = (size_t)(row0 + r_lo + ti) * hq + (size_t)g * G + h;
+      uint4* dst = reinterpret_cast<uint4*>(out + head * kD);
 #pragma unroll
       for (int c = 0; c < kD / 32; ++c) {
         uint32_t v[32];
         tc_ld32(lane_base + COL_O + c * 32, v);
         tc_wait_ld();
-        if (row_ok) {
+        if (row_ok && gate.g) {  // fused output gate: O = g A + (1 - g) X, one rounding
+#pragma unroll
+          for (int xx = 0; xx < 32; ++xx)
+            v[xx] = __float_as_uint(gate_apply<bf16>(gate, head, c * 32 + xx, kD,
+                                                     __uint_as_float(v[xx]) * inv));
+#pragma unroll
+          for (int xx = 0; xx < 32; xx += 8) {
+            uint4 w;
+            w.x = pack_bf16(__uint_as_float(v[xx]), __uint_as_float(v[xx + 1]));
+            w.y = pack_bf16(__uint_as_float(v[xx + 2]), __uint_as_float(v[xx + 3]));
+            w.z = pack_bf16(__uint_as_float(v[xx + 4]), __uint_as_float(v[xx + 5]));
+            w.w = pack_bf16(__uint_as_float(v[xx + 6]), __uint_as_float(v[xx + 7]));
+            dst[(c * 32 + xx) / 8] = w;
+          }
+        } else if (row_ok) {
 #pragma unroll
           for (int xx = 0; xx < 32; xx += 8) {
             uint4 w;
@@ -632,7 +646,7 @@ template <int B, int G>
 static cudaError_t launch_tc(const msa_paged_kv_t* kv, const CUtensorMap& tk, const CUtensorMap& tv,
                              const void* q, const int32_t* cu_q, int units, int ups, int ecap,
                              const int2* entries, const int* counts, float sl2, void* out,
-                             float* lse, cudaStream_t st) {
+                             float* lse, gate_t gate, cudaStream_t st) {
   constexpr int NST = (B == 128) ? 3 : 4;
   const size_t smem = (size_t)NST * 2 * B * kD * 2 + 1024;
   auto kern = prefill_tc_kernel<B, G>;
@@ -641,13 +655,13 @@ static cudaError_t launch_tc(const msa_paged_kv_t* kv, const CUtensorMap& tk, co
   kern<<<units, 192, smem, st>>>(tk, tv, (const bf16*)q, cu_q, kv->page_table, kv->seq_lens,
                                  kv->status_word, kv->num_q_heads, kv->num_kv_heads, kv->num_pages,
                                  kv->max_blocks_per_seq, ups, ecap, entries, counts, sl2,
-                                 (bf16*)out, lse);
+                                 (bf16*)out, lse, gate);
   return cudaGetLastError();
 }
 
 cudaError_t prefill_tc(const msa_paged_kv_t* kv, const void* q, const int32_t* cu_q, int max_rows,
                        const int32_t* idx, int top_k, float scale, void* out, float* lse, void* ws,
-                       cudaStream_t st) {
+                       gate_t gate, cudaStream_t st) {
   const int G = kv->num_q_heads / kv->num_kv_heads, B = kv->block_size;
   const int TM = 128 / G;
   int ups;
@@ -667,10 +681,10 @@ cudaError_t prefill_tc(const msa_paged_kv_t* kv, const void* q, const int32_t* c
     return cudaErrorInvalidValue;
   const float sl2 = scale * kLog2e;
   if (B == 128)
-    return G == 8 ? launch_tc<128, 8>(kv, tk, tv, q, cu_q, units, ups, ecap, entries, counts, sl2, out, lse, st)
-                  : launch_tc<128, 16>(kv, tk, tv, q, cu_q, units, ups, ecap, entries, counts, sl2, out, lse, st);
-  return G == 8 ? launch_tc<64, 8>(kv, tk, tv, q, cu_q, units, ups, ecap, entries, counts, sl2, out, lse, st)
-                : launch_tc<64, 16>(kv, tk, tv, q, cu_q, units, ups, ecap, entries, counts, sl2, out, lse, st);
+    return G == 8 ? launch_tc<128, 8>(kv, tk, tv, q, cu_q, units, ups, ecap, entries, counts, sl2, out, lse, gate, st)
+                  : launch_tc<128, 16>(kv, tk, tv, q, cu_q, units, ups, ecap, entries, counts, sl2, out, lse, gate, st);
+  return G == 8 ? launch_tc<64, 8>(kv, tk, tv, q, cu_q, units, ups, ecap, entries, counts, sl2, out, lse, gate, st)
+                : launch_tc<64, 16>(kv, tk, tv, q, cu_q, units, ups, ecap, entries, counts, sl2, out, lse, gate, st);
 }
 
 }  // namespace msa

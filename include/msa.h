@@ -209,6 +209,47 @@ msa_status_t msa_sparse_attn_decode(const msa_paged_kv_t* kv, const void* q,
                                     msa_stream_t stream);
 
 /*
+ * msa_sparse_attn_prefill_gated / msa_sparse_attn_decode_gated - the two
+ * attention calls above with the output gate fused into their epilogues:
+ *
+ *   O = g * A + (1 - g) * X
+ *
+ * where A is the sparse attention output. Follows "Sparse Attention for
+ * Long-Context LLMs: Evolution and Practical Deployment", section 4.3 (step 6
+ * of the computation flow: the gate weights the sparse attention output
+ * against the original representation; it may be a scalar or vary with the
+ * dimension). The gate values are the caller's (a learned gate is applied
+ * before the call); the library does not compute them. A is not rounded
+ * before the gate: the result is rounded to kv->dtype once.
+ *
+ *   gate          : device fp32, [rows][num_q_heads] (gate_per_dim = 0: one
+ *                   value per row and head) or [rows][num_q_heads][head_dim]
+ *                   (gate_per_dim = 1); rows = num_rows (prefill) or batch
+ *                   (decode). 4-byte aligned.
+ *   x             : device [rows][num_q_heads][head_dim] in kv->dtype, the
+ *                   other branch (the query itself, or a residual). 16-byte
+ *                   aligned. May alias q, not out.
+ *   lse           : the attention's log-sum-exp, not gated.
+ *   other arguments, workspace and errors: as for the ungated calls;
+ *   MSA_ERR_INVALID_ARG also for a NULL or misaligned gate or x, or
+ *   gate_per_dim not 0 or 1.
+ */
+msa_status_t msa_sparse_attn_prefill_gated(const msa_paged_kv_t* kv, const void* q,
+                                           const int32_t* cu_q, int32_t num_rows,
+                                           int32_t max_rows_per_seq, const int32_t* block_idx,
+                                           int32_t top_k, float softmax_scale, const float* gate,
+                                           int32_t gate_per_dim, const void* x, void* out,
+                                           float* lse, void* workspace, size_t workspace_bytes,
+                                           msa_stream_t stream);
+
+msa_status_t msa_sparse_attn_decode_gated(const msa_paged_kv_t* kv, const void* q,
+                                          const int32_t* block_idx, int32_t top_k,
+                                          float softmax_scale, const float* gate,
+                                          int32_t gate_per_dim, const void* x, void* out,
+                                          float* lse, void* workspace, size_t workspace_bytes,
+                                          msa_stream_t stream);
+
+/*
  * msa_sparse_attn_decode_noalloc - msa_sparse_attn_decode for callers that
  * cannot allocate device memory at the call: a plugin run by a host framework
  * that owns the device memory pool and offers no scratch allocator, or a

@@ -24,6 +24,10 @@ Citations (page title, section):
   * attend     - "MiniMax Sparse Attention", method paragraph (exact blockwise
                  sparse attention over the chosen blocks) and "Sparse Attention
                  + Linear Backbones", section 5.5 (softmax(q k^T / sqrt(d)) v).
+  * gate       - "Sparse Attention for Long-Context LLMs: Evolution and
+                 Practical Deployment", section 4.3, step 6 of the computation
+                 flow: O = Gate * A + (1 - Gate) * X, the gate a scalar or
+                 varying with the dimension (X given by the caller).
 """
 from __future__ import annotations
 
@@ -156,3 +160,28 @@ def forward(Q, K, V, pos, block: int, top_k: int, scale: float) -> Dict[str, np.
     idx, gap = select(S, pos, block, top_k)
     O, lse = attend(Q, K, V, pos, idx, block, scale)
     return {"centroids": C, "scores": S, "idx": idx, "gap": gap, "out": O, "lse": lse}
+
+
+def gate(A, g, X) -> np.ndarray:
+    """O = g * A + (1 - g) * X in fp64, literally. A, X: [R, Hq, d]; g: [R, Hq]
+    (one value per row and head) or [R, Hq, d]."""
+    A = np.asarray(A, dtype=np.float64)
+    X = np.asarray(_widen(X), dtype=np.float64)
+    g = np.asarray(g, dtype=np.float64)
+    if g.ndim == A.ndim - 1:
+        g = g[..., None]
+    return g * A + (1.0 - g) * X
+
+
+def _widen(x):
+    """bf16 torch tensors / uint16 bit patterns -> float64 values."""
+    try:
+        import torch
+        if isinstance(x, torch.Tensor):
+            return x.detach().to("cpu").double().numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    x = np.asarray(x)
+    if x.dtype == np.uint16:
+        return (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    return x.astype(np.float64)

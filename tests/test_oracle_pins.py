@@ -264,3 +264,32 @@ def test_tiny_workload_finds_planted_blocks():
     S = r["scores"][0, 0, :L // w.block - 1]
     assert sorted(np.argsort(-S)[:2].tolist()) == planted
     assert set(planted) <= set(int(j) for j in r["idx"][0, 0])
+
+
+# ---------------------------------------------------------------------------
+# output gate: O = g * A + (1 - g) * X
+# ---------------------------------------------------------------------------
+def test_gate_special_cases_and_broadcast():
+    rng = np.random.default_rng(5)
+    A = rng.standard_normal((3, 4, 8))
+    X = rng.standard_normal((3, 4, 8))
+    one, zero = np.ones((3, 4)), np.zeros((3, 4))
+    assert np.array_equal(oracle.gate(A, one, X), A)        # g = 1: attention only
+    assert np.array_equal(oracle.gate(A, zero, X), X)       # g = 0: the other branch only
+    half = oracle.gate(A, np.full((3, 4), 0.5), X)
+    assert np.allclose(half, (A + X) / 2, rtol=0, atol=1e-15)
+    # a per-head gate equals the same value repeated over the coordinates
+    g = rng.uniform(0, 1, (3, 4))
+    assert np.allclose(oracle.gate(A, g, X), oracle.gate(A, np.repeat(g[..., None], 8, -1), X),
+                       rtol=0, atol=1e-15)
+    # per-coordinate gate: coordinate c of head h uses g[.., h, c] (catches a transposed gate)
+    gd = rng.uniform(0, 1, (3, 4, 8))
+    r, h, c = 2, 1, 5
+    assert oracle.gate(A, gd, X)[r, h, c] == gd[r, h, c] * A[r, h, c] + (1 - gd[r, h, c]) * X[r, h, c]
+
+
+def test_gate_widens_bf16_branch():
+    x = torch.tensor([[[1.5, -2.25]]], dtype=torch.bfloat16)
+    A = np.array([[[0.5, 0.25]]])
+    out = oracle.gate(A, np.array([[0.25]]), x)
+    assert np.array_equal(out, 0.25 * A + 0.75 * np.array([[[1.5, -2.25]]]))
