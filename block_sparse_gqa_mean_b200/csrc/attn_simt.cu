@@ -127,7 +127,8 @@ __global__ void __launch_bounds__(128) attn_simt_kernel(
   for (int e = tid; e < G * D; e += blockDim.x) {
     const int h = e / D;
     out[((size_t)row * hq + g * G) * D + e] = from_f32<T>(
-        gate_apply<T>(gate, (size_t)row * hq + g * G + h, e - h * D, D, os[e] / l_s[h]));
+        gate_apply<T>(gate, (size_t)row * hq + g * G + h, e - h * D, D,
+                      l_s[h] > 0.f ? os[e] / l_s[h] : 0.f));  // no key: A = 0
   }
   if (lse && tid < G) lse[(size_t)row * hq + g * G + tid] = m_s[tid] + logf(l_s[tid]);
 }

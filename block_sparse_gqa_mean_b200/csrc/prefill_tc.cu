@@ -31,7 +31,7 @@
 // double-buffered and the softmax reference max moves lazily (only when a
 // row's max grows by more than 2^8), so writing P never waits for the P V in
 // flight and O is rescaled in TMEM only rarely.
-#include "tma.cuh"
+#include "tc.cuh"
 
 namespace msa {
 
@@ -39,98 +39,6 @@ namespace {
 
 constexpr int kD = 128;
 constexpr float kLog2e = 1.4426950408889634f;
-
-
-// ---- tcgen05 wrappers ------------------------------------------------------
-__device__ __forceinline__ void tc_fence_before() {
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-
-// A from TMEM, B from shared memory (descriptor), D in TMEM.
-__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                          uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n"
-      " .reg .pred p;\n"
-      " setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %5, %5, %5}, p;\n"
-      "}\n" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0u));
-}
-
-__device__ __forceinline__ void tc_commit(uint64_t* bar) {
-  asm volatile(
-      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-          smem_u32(bar))
-      : "memory");
-}
-
-__device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-__device__ __forceinline__ void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
-
-// 32 lanes x 32 consecutive 32-bit columns: thread i of the warp gets lane i.
-__device__ __forceinline__ void tc_ld32(uint32_t taddr, uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
-      "%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
-        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
-        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr));
-}
-
-__device__ __forceinline__ void tc_st32(uint32_t taddr, const uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
-      "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
-      "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
-      "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
-      "r"(r[29]), "r"(r[30]), "r"(r[31])
-      : "memory");
-}
-
-__device__ __forceinline__ void tc_ld1(uint32_t taddr, uint32_t (&r)[1]) {
-  asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r[0]) : "r"(taddr));
-}
-__device__ __forceinline__ void tc_st1(uint32_t taddr, const uint32_t (&r)[1]) {
-  asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(r[0]) : "memory");
-}
-
-// Shared-memory matrix descriptor, 128-byte swizzle (sm_100 layout: start
-// address, leading and stride byte offsets in 16-byte units, version 1).
-__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
-  uint64_t d = 0;
-  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
-  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
-  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
-  d |= (uint64_t)1 << 46;
-  d |= (uint64_t)2 << 61;
-  return d;
-}
-
-// Instruction descriptor, kind::f16: bf16 A and B, fp32 D, M x N.
-__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) |
-         ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
-}
-
-__device__ __forceinline__ float fast_exp2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&v);
-}
 
 }  // namespace
 
@@ -220,52 +128,84 @@ __global__ void __launch_bounds__(128) prefill_plan_kernel(
 // ---------------------------------------------------------------------------
 constexpr float kRescaleLog2 = 8.f;  // lazy rescale threshold (log2 units)
 
-__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
-  return ((uint64_t)__float_as_uint(hi) << 32) | __float_as_uint(lo);
-}
-__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
-__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
+
+// 2 NP scores -> NP bf16 pairs P = exp2(s * c - m) and their fp32 sum (of the
+// rounded values) added into lsum2 (two partial sums). One pair in four on
+// the FMA pipe, the rest on MUFU.
+template <int NP>
+__device__ __forceinline__ void exp_pack(const float* s, uint64_t sl2, uint64_t neg_m,
+                                         uint32_t (&pv)[NP], uint64_t& lsum2) {
+#pragma unroll
+  for (int xx = 0; xx < NP; ++xx) {
+    const uint64_t arg = f2_fma(f2_pack(s[2 * xx], s[2 * xx + 1]), sl2, neg_m);
+    if ((xx & 3) == 0) {
+      float p0, p1;
+      exp2_poly_pair(arg, p0, p1);
+      pv[xx] = pack_bf16(p0, p1);
+    } else {
+      pv[xx] = pack_bf16(fast_exp2(__uint_as_float((uint32_t)arg)),
+                         fast_exp2(__uint_as_float((uint32_t)(arg >> 32))));
+    }
+    // the rounded pair, widened back to fp32, into the row sum
+    lsum2 = f2_add(lsum2, ((uint64_t)(pv[xx] & 0xffff0000u) << 32) | (uint64_t)(pv[xx] << 16));
+  }
 }
 
-// 2^x for two lanes on the FMA pipe, to share the exponentials with the
-// MUFU unit. x is clamped to [-120, +inf); rint(x) comes from adding
-// 1.5 * 2^23 (the sum's low mantissa bits hold rint(x)), f = x - rint(x) lies
-// in [-0.5, 0.5], 2^f is a cubic minimax fit (relative error 7.5e-5, fitted
-// for this kernel by a Remez exchange on relative error), and rint(x) is
-// added to the exponent field. The result is rounded to bf16 afterwards.
-constexpr uint32_t kMagic = 0x4B400000u;  // 1.5 * 2^23
-__device__ __forceinline__ void exp2_poly_pair(uint64_t arg, float& r0, float& r1) {
-  constexpr uint64_t MAGIC = ((uint64_t)kMagic << 32) | kMagic;
-  constexpr uint64_t NMAGIC = ((uint64_t)(kMagic | 0x80000000u) << 32) | (kMagic | 0x80000000u);
-  constexpr uint64_t NEG1 = 0xBF800000BF800000ull;
-  constexpr uint64_t C0 = 0x3F7FFB49'3F7FFB49ull;   // 9.999280572e-01
-  constexpr uint64_t C1 = 0x3F31798D'3F31798Dull;   // 6.932609677e-01
-  constexpr uint64_t C2 = 0x3E786F0D'3E786F0Dull;   // 2.426111251e-01
-  constexpr uint64_t C3 = 0x3D61FBB0'3D61FBB0ull;   // 5.517166853e-02
-  const float x0 = fmaxf(__uint_as_float((uint32_t)arg), -120.f);
-  const float x1 = fmaxf(__uint_as_float((uint32_t)(arg >> 32)), -120.f);
-  const uint64_t X = f2_pack(x0, x1);
-  const uint64_t T = f2_add(X, MAGIC);
-  const uint64_t J = f2_add(T, NMAGIC);
-  const uint64_t F = f2_fma(J, NEG1, X);
-  uint64_t P = f2_fma(F, C3, C2);
-  P = f2_fma(P, F, C1);
-  P = f2_fma(P, F, C0);
-  r0 = __int_as_float((int)(uint32_t)P + ((int)(uint32_t)T << 23));
-  r1 = __int_as_float((int)(uint32_t)(P >> 32) + ((int)(uint32_t)(T >> 32) << 23));
+// 16 lanes x 2N columns in two halves: thread t < 16 reads lane (base + t),
+// columns 0..N-1 of the address; thread t >= 16 reads lane (base + t - 16),
+// columns N..2N-1.
+__device__ __forceinline__ void tc_ld16x2(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x32bx2.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
+      "%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32], 32;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tc_ld16x2(uint32_t taddr, uint32_t (&r)[64]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x32bx2.x64.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
+      "%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,"
+      "%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,"
+      "%61,%62,%63}, [%64], 64;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]),
+        "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]),
+        "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]),
+        "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]),
+        "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]),
+        "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]),
+        "=r"(r[62]), "=r"(r[63])
+      : "r"(taddr));
 }
 
-__device__ __forceinline__ float max3(float a, float b, float c) {
-  float d;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
-  return d;
+// 16 lanes x 2N columns in two halves: thread t < 16 writes lane (base + t),
+// columns 0..N-1; thread t >= 16 writes lane (base + t - 16), columns N..2N-1.
+__device__ __forceinline__ void tc_st16x2(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x32bx2.x16.b32 [%0], 16, {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
+      "%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15])
+      : "memory");
+}
+__device__ __forceinline__ void tc_st16x2(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x32bx2.x32.b32 [%0], 32, {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
+      "%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
+      "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
+      "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
 }
 
 template <int B, int G>
@@ -446,10 +386,28 @@ __global__ void __launch_bounds__(192, 1) prefill_tc_kernel(
     // m_ref moves, and O, l are rescaled, only when a row's max exceeds m_ref by
     // more than kRescaleLog2, so the weights stay below 2^8 and writing P never
     // has to wait for the P*V in flight. Rows whose token did not select the
-    // block use m = +inf, which turns every weight into an exact 0.
+    // block get zero weights.
+    //
+    // A warp holds 32 rows = 32 / G tokens, split into two halves of 16 TMEM
+    // lanes. When the block was selected only by tokens of one half, the warp
+    // works on that half alone: a 16-lane access (16x32bx2) gives each of the
+    // half's rows to two threads, 64 columns each (thread t: row 16*half +
+    // t % 16, columns 64 * (t / 16) ..), so the exponentials of the block cost
+    // half as much; the row's max and sum are combined over the thread pair,
+    // and its state (m_ref, l_run) stays with the thread that owns the row.
     float m_ref = -INFINITY;
     float l_run = 0.f;  // row sum of the bf16-rounded weights P (the ones P V uses)
     const uint64_t sl2 = f2_pack(scale_log2, scale_log2);
+    // the row this thread works on when only half hv (0, 1) of the warp is busy
+    int ti_half[2], t_half[2];
+    bool ok_half[2];
+#pragma unroll
+    for (int hv = 0; hv < 2; ++hv) {
+      ti_half[hv] = (quarter * 32 + hv * 16 + (lane & 15)) / G;
+      ok_half[hv] = ti_half[hv] < nr;
+      t_half[hv] = t_first + ti_half[hv];
+    }
+    const bool upper = lane >= 16;  // which 64 columns of the half-mode row
     int2 en_next = ent[0];
     for (int e = 0; e < n_e; ++e) {
       if (__any_sync(0xffffffffu, s_abort != 0)) break;
@@ -463,10 +421,17 @@ __global__ void __launch_bounds__(192, 1) prefill_tc_kernel(
       tc_fence_after();
       const int j = en.x;
       const bool sel = row_ok && ((en.y >> ti) & 1);
-      const bool warp_sel = __any_sync(0xffffffffu, sel);
-      const int kmax = t - j * B;  // visible keys: index <= kmax
+      const uint32_t bal = __ballot_sync(0xffffffffu, sel);
+      // 0: no row, 1: one half (hv), 2: both halves
+      const int mode = (bal == 0u) ? 0 : (((bal & 0xffffu) != 0u) && ((bal >> 16) != 0u)) ? 2 : 1;
+      const int hv = (bal & 0xffffu) ? 0 : 1;
+      const bool owner = upper == (hv == 1);       // half mode: this thread's own row is the half's row
+      // half-mode row of this thread and its visible keys
+      const int kmax_h = (hv ? t_half[1] : t_half[0]) - j * B - (upper ? B / 2 : 0);
+      const bool sel_h = (hv ? ok_half[1] : ok_half[0]) && ((en.y >> (hv ? ti_half[1] : ti_half[0])) & 1);
+      const int kmax = t - j * B;  // full mode: visible keys of this thread's row: index <= kmax
       float s[B];
-      if (warp_sel) {
+      if (mode == 2) {
 #pragma unroll
         for (int c = 0; c < B / 32; ++c) {
           uint32_t v[32];
@@ -475,12 +440,18 @@ __global__ void __launch_bounds__(192, 1) prefill_tc_kernel(
           for (int xx = 0; xx < 32; ++xx) s[c * 32 + xx] = __uint_as_float(v[xx]);
         }
         tc_wait_ld();
+      } else if (mode == 1) {
+        uint32_t v[B / 2];
+        tc_ld16x2(lane_base + ((uint32_t)(hv * 16) << 16) + COL_S, v);
+#pragma unroll
+        for (int xx = 0; xx < B / 2; ++xx) s[xx] = __uint_as_float(v[xx]);
+        tc_wait_ld();
       }
       tc_fence_before();
       mbar_arrive(&s_free);                        // S is in registers: the next S may start
 
-      float mraw = -INFINITY;                      // max of the raw scores
-      if (warp_sel) {
+      float mraw = -INFINITY;                      // max of the raw scores of this thread's row
+      if (mode == 2) {
         if (__any_sync(0xffffffffu, kmax < B - 1)) {
           // a block that holds some row's own position: mask keys after it
 #pragma unroll
@@ -493,10 +464,23 @@ __global__ void __launch_bounds__(192, 1) prefill_tc_kernel(
           for (int a = 0; a < 4; ++a) m4[a] = max3(m4[a], s[c + 2 * a], s[c + 2 * a + 1]);
         }
         mraw = max3(m4[0], m4[1], fmaxf(m4[2], m4[3]));
+      } else if (mode == 1) {
+        if (__any_sync(0xffffffffu, kmax_h < B / 2 - 1)) {
+#pragma unroll
+          for (int c = 0; c < B / 2; ++c) s[c] = (c <= kmax_h) ? s[c] : -INFINITY;
+        }
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int c = 0; c < B / 2; c += 8) {
+#pragma unroll
+          for (int a = 0; a < 4; ++a) m4[a] = max3(m4[a], s[c + 2 * a], s[c + 2 * a + 1]);
+        }
+        const float mh = max3(m4[0], m4[1], fmaxf(m4[2], m4[3]));
+        mraw = fmaxf(mh, __shfl_xor_sync(0xffffffffu, mh, 16));  // both halves of the row
       }
       bool rescale = false;
       float alpha = 1.f;
-      if (sel) {
+      if (sel) {  // this thread's own row (in half mode its owner has the pair's max)
         const float mx = mraw * scale_log2;
         if (m_ref == -INFINITY) {
           m_ref = mx;                              // first block of this row: O and l are zero
@@ -531,43 +515,50 @@ __global__ void __launch_bounds__(192, 1) prefill_tc_kernel(
       const int pb = e & 1;
       // P = exp2(s*c - m_ref) rounded to bf16 (the tensor cores sum the same
       // rounded weights into l, so the output is an exact convex combination)
-      const float m_use = sel ? m_ref : INFINITY;
-      const uint64_t neg_m = f2_pack(-m_use, -m_use);
-      uint64_t lsum2 = 0ull;  // two fp32 partial sums
+      const float m_own = sel ? m_ref : INFINITY;
+      if (mode == 2) {
+        const uint64_t neg_m = f2_pack(-m_own, -m_own);
+        uint64_t lsum2 = 0ull;  // two fp32 partial sums
 #pragma unroll
-      for (int cc = 0; cc < B / 64; ++cc) {
-        uint32_t pv[32];
-        if (warp_sel) {
-#pragma unroll
-          for (int xx = 0; xx < 32; ++xx) {
-            const uint64_t arg = f2_fma(f2_pack(s[64 * cc + 2 * xx], s[64 * cc + 2 * xx + 1]), sl2, neg_m);
-            if ((xx & 3) == 0) {  // one pair in four on the FMA pipe, the rest on MUFU
-              float p0, p1;
-              exp2_poly_pair(arg, p0, p1);
-              pv[xx] = pack_bf16(p0, p1);
-            } else {
-              pv[xx] = pack_bf16(fast_exp2(__uint_as_float((uint32_t)arg)),
-                                 fast_exp2(__uint_as_float((uint32_t)(arg >> 32))));
-            }
-            // the rounded pair, widened back to fp32, into the row sum
-            lsum2 = f2_add(lsum2, ((uint64_t)(pv[xx] & 0xffff0000u) << 32) | (uint64_t)(pv[xx] << 16));
-          }
-        } else {
-#pragma unroll
-          for (int xx = 0; xx < 32; ++xx) pv[xx] = 0u;
+        for (int cc = 0; cc < B / 64; ++cc) {
+          uint32_t pv[32];
+          exp_pack<32>(s + 64 * cc, sl2, neg_m, pv, lsum2);
+          tc_st32(lane_base + COL_P + pb * 64 + cc * 32, pv);
         }
-        tc_st32(lane_base + COL_P + pb * 64 + cc * 32, pv);
+        l_run += __uint_as_float((uint32_t)lsum2) + __uint_as_float((uint32_t)(lsum2 >> 32));
+      } else if (mode == 1) {
+        // the half's rows: m from the row's owner; the other half's rows: zero weights
+        const float m_pair = __shfl_xor_sync(0xffffffffu, m_own, 16);
+        const float m_use = owner ? m_own : m_pair;
+        const float mu = sel_h ? m_use : INFINITY;
+        const uint64_t neg_m = f2_pack(-mu, -mu);
+        uint64_t lsum2 = 0ull;
+        uint32_t pv[B / 4];
+        exp_pack<B / 4>(s, sl2, neg_m, pv, lsum2);
+        tc_st16x2(lane_base + ((uint32_t)(hv * 16) << 16) + COL_P + pb * 64, pv);
+#pragma unroll
+        for (int xx = 0; xx < B / 4; ++xx) pv[xx] = 0u;
+        tc_st16x2(lane_base + ((uint32_t)((1 - hv) * 16) << 16) + COL_P + pb * 64, pv);
+        const float lh = __uint_as_float((uint32_t)lsum2) + __uint_as_float((uint32_t)(lsum2 >> 32));
+        const float lp = __shfl_xor_sync(0xffffffffu, lh, 16);
+        if (owner && sel) l_run += lh + lp;
+      } else {
+        uint32_t pv[32];
+#pragma unroll
+        for (int xx = 0; xx < 32; ++xx) pv[xx] = 0u;
+#pragma unroll
+        for (int cc = 0; cc < B / 64; ++cc) tc_st32(lane_base + COL_P + pb * 64 + cc * 32, pv);
       }
       tc_wait_st();
       tc_fence_before();
       mbar_arrive(&p_full[pb]);
-      l_run += __uint_as_float((uint32_t)lsum2) + __uint_as_float((uint32_t)(lsum2 >> 32));
     }
     // epilogue: O / l -> bf16 once the last P*V has completed
     const bool go = !__any_sync(0xffffffffu, s_abort != 0);
     if (go && __all_sync(0xffffffffu, mbar_wait(&o_done[(n_e - 1) & 1], ((n_e - 1) >> 1) & 1))) {
       tc_fence_after();
-      const float l = l_run;
+      // a row that took no block (its token selected none) has an empty sum: A = 0
+      const float l = (m_ref == -INFINITY) ? 0.f : l_run;
       const float inv = (l > 0.f) ? 1.f / l : 0.f;
       const size_t head = (size_t)(row0 + r_lo + ti) * hq + (size_t)g * G + h;
       uint4* dst = reinterpret_cast<uint4*>(out + head * kD);

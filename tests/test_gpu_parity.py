@@ -186,6 +186,88 @@ def test_chunked_prefill_matches_full():
     compare(out, full[4][T0:].float().cpu().double().numpy(), "bf16")
 
 
+def test_prefill_batch_varlen_chunked_and_index_edges():
+    """Three sequences in one call: a full prefill of 700 rows, a chunk of 900
+    rows after 1000 cached tokens, and 2600 rows (ragged last query tiles); then
+    the same call with a repeated block in some rows (counted once) and rows
+    without any block (A = 0, lse = -inf)."""
+    w = workloads.prefill_bf16(batch=3, ctx=(700, 1900, 2600), top_k=8)
+    p = workloads.paging(w)
+    cache = new_cache(w, p)
+    first = [0, 1000, 0]
+    append(cache, w, [0, 0, 0], first)
+    append(cache, w, first, list(w.ctx))
+    n = [w.ctx[b] - first[b] for b in range(3)]
+    q = torch.cat([workloads.queries_prefill(w, b, first[b], w.ctx[b], DEV) for b in range(3)])
+    cu = msa.cu_seqlens(n, DEV)
+    idx, _ = msa.select_topk(cache, q, w.top_k, cu_q=cu, max_rows_per_seq=max(n))
+    out, lse = msa.sparse_attn_prefill(cache, q, idx, cu_q=cu, max_rows_per_seq=max(n))
+    # edge rows: slot 1 repeats slot 0 (the oracle gets -1 there), or no block at all
+    rng = np.random.default_rng(7)
+    idx_e = idx.cpu().numpy().copy()
+    ref_e = idx_e.copy()
+    rows = rng.choice(len(idx_e), 300, replace=False)
+    dup, empty = rows[:200], rows[200:]
+    for r in dup:
+        g = int(rng.integers(w.hkv))
+        if idx_e[r, g, 1] >= 0:
+            idx_e[r, g, 1] = idx_e[r, g, 0]
+            ref_e[r, g, 1] = -1
+    idx_e[empty] = -1
+    ref_e[empty] = -1
+    out_e, lse_e = msa.sparse_attn_prefill(cache, q, torch.from_numpy(idx_e).to(DEV), cu_q=cu,
+                                           max_rows_per_seq=max(n))
+    torch.cuda.synchronize()
+    assert cache.device_status() == 0
+    gi = idx.cpu().numpy()
+    r0 = 0
+    for b in range(3):
+        pos = np.arange(first[b], w.ctx[b])
+        sl = slice(r0, r0 + n[b])
+        qb = q[sl].cpu()
+        orc = oracle_rows(w, b, w.ctx[b], pos, qb, idx=gi[sl])
+        compare(out[sl], orc["out"], w.dtype)
+        assert np.abs(lse[sl].cpu().double().numpy() - orc["lse"]).max() < 2e-3
+        orc_e = oracle_rows(w, b, w.ctx[b], pos, qb, idx=ref_e[sl])
+        keep = ~np.isin(np.arange(r0, r0 + n[b]), empty)
+        compare(out_e[sl][torch.from_numpy(keep).to(DEV)], orc_e["out"][keep], w.dtype)
+        le = lse_e[sl].cpu().double().numpy()
+        assert np.abs(le[keep] - orc_e["lse"][keep]).max() < 2e-3
+        r0 += n[b]
+    assert torch.all(out_e[torch.from_numpy(empty).to(DEV)] == 0)
+    assert torch.all(torch.isneginf(lse_e[torch.from_numpy(empty).to(DEV)]))
+
+
+EMPTY_CASES = [("g8_b128", dict(ctx=(700,), top_k=4)),
+               ("g16_b128", dict(ctx=(600,), hq=64, hkv=4, top_k=3)),
+               ("g8_b64", dict(ctx=(500,), block=64, top_k=5)),
+               ("g4_simt", dict(ctx=(400,), hq=16, hkv=4, top_k=3))]
+
+
+@pytest.mark.parametrize("name,over", EMPTY_CASES, ids=[c[0] for c in EMPTY_CASES])
+def test_rows_without_blocks(name, over):
+    """A row whose block list is all -1 attends to nothing: A = 0, lse = -inf,
+    on every prefill path; the other rows are unaffected."""
+    w = workloads.prefill_bf16(**over)
+    cache = new_cache(w, workloads.paging(w))
+    T = w.ctx[0]
+    append(cache, w, [0], [T])
+    q = workloads.queries_prefill(w, 0, 0, T, DEV)
+    cu = msa.cu_seqlens([T], DEV)
+    idx, _ = msa.select_topk(cache, q, w.top_k, cu_q=cu, max_rows_per_seq=T)
+    ref, ref_lse = msa.sparse_attn_prefill(cache, q, idx, cu_q=cu, max_rows_per_seq=T)
+    empty = torch.arange(3, T, 7, device=DEV)
+    idx2 = idx.clone()
+    idx2[empty] = -1
+    out, lse = msa.sparse_attn_prefill(cache, q, idx2, cu_q=cu, max_rows_per_seq=T)
+    torch.cuda.synchronize()
+    assert cache.device_status() == 0
+    assert torch.all(out[empty] == 0) and torch.all(torch.isneginf(lse[empty]))
+    keep = torch.ones(T, dtype=torch.bool, device=DEV)
+    keep[empty] = False
+    assert torch.equal(out[keep].view(torch.int16), ref[keep].view(torch.int16))
+
+
 # ---------------------------------------------------------------------------
 # decode
 # ---------------------------------------------------------------------------
