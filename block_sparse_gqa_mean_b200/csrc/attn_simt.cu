@@ -65,7 +65,7 @@ __global__ void __launch_bounds__(128) attn_simt_kernel(
   const int32_t* sel = block_idx + ((size_t)row * hkv + g) * top_k;
   for (int s = 0; s < top_k; ++s) {
     const int j = sel[s];
-    if (j < 0) continue;
+    if (j < 0 || (s > 0 && j == sel[s - 1])) continue;  // a repeated block counts once
     if (j > own) {
       if (tid == 0) report(status, MSA_DEV_BAD_INDEX);
       continue;

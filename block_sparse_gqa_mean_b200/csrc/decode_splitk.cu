@@ -108,6 +108,8 @@ __global__ void __launch_bounds__(128) decode_splitk_kernel(
     bool ok = false;
     if (base + tid < nslots) {
       j = sel[base + tid];
+      // a block repeated in the adjacent slot (rows are ascending) counts once
+      if (j >= 0 && s0 + base + tid > 0 && sel[base + tid - 1] == j) j = -1;
       if (j >= 0) {
         if (j > t / B) {
           report(status, MSA_DEV_BAD_INDEX);

@@ -178,7 +178,10 @@ msa_status_t msa_select_topk(const msa_paged_kv_t* kv, const void* q, const int3
  *                       not be NULL here).
  *   block_idx         : device [num_rows][num_kv_heads][top_k] int32, as
  *                       produced by msa_select_topk (ascending, -1 padded,
- *                       every entry <= t / B).
+ *                       every entry <= t / B). U is a set: a block repeated
+ *                       in the adjacent slot counts once; a row without any
+ *                       block gives out = 0 (A = 0 before a gate) and
+ *                       lse = -inf.
  *   out               : device [num_rows][num_q_heads][head_dim], kv->dtype.
  *   lse               : device [num_rows][num_q_heads] fp32, or NULL.
  *   workspace         : device scratch, msa_workspace_size(MSA_OP_PREFILL, ..).
@@ -199,7 +202,9 @@ msa_status_t msa_sparse_attn_prefill(const msa_paged_kv_t* kv, const void* q, co
  * above.
  *
  *   q                 : device [batch][num_q_heads][head_dim], kv->dtype.
- *   block_idx         : device [batch][num_kv_heads][top_k] int32.
+ *   block_idx         : device [batch][num_kv_heads][top_k] int32, the same
+ *                       rules as for prefill (ascending, -1 padded, an
+ *                       adjacent repeat counts once, an empty row gives 0).
  *   out, lse          : device [batch][num_q_heads][head_dim] / [batch][num_q_heads].
  *   workspace         : device scratch, msa_workspace_size(MSA_OP_DECODE, ..).
  */

@@ -135,7 +135,8 @@ void orc_select(const double* S, int64_t R, const int64_t* pos, int hkv, int64_t
 // Exact attention over the selected blocks. For row r, head h (group g):
 // keys u of the listed blocks with u <= pos[r] and u < L; logits
 // l_u = scale * q . k_u; w = softmax(l); O = sum_u w_u v_u; lse = log sum exp(l).
-// idx entries < 0 are padding; entries may come in any order.
+// idx entries < 0 are padding; entries may come in any order. The attended
+// tokens form a set, so a block listed twice in a row counts once.
 void orc_attend(const void* Q, const void* K, const void* V, int dtype, int64_t R,
                 const int64_t* pos, int64_t L, int hq, int hkv, int d, int B, const int32_t* idx,
                 int k, double scale, double* O, double* lse) {
@@ -148,6 +149,9 @@ void orc_attend(const void* Q, const void* K, const void* V, int dtype, int64_t 
       std::vector<int64_t> keys_u;
       for (int s = 0; s < k; ++s) {
         if (blocks[s] < 0) continue;
+        bool seen = false;
+        for (int s2 = 0; s2 < s; ++s2) seen = seen || blocks[s2] == blocks[s];
+        if (seen) continue;
         for (int64_t u = (int64_t)blocks[s] * B; u < (int64_t)(blocks[s] + 1) * B; ++u)
           if (u <= pos[r] && u < L) keys_u.push_back(u);
       }

@@ -202,19 +202,17 @@ def test_prefill_batch_varlen_chunked_and_index_edges():
     cu = msa.cu_seqlens(n, DEV)
     idx, _ = msa.select_topk(cache, q, w.top_k, cu_q=cu, max_rows_per_seq=max(n))
     out, lse = msa.sparse_attn_prefill(cache, q, idx, cu_q=cu, max_rows_per_seq=max(n))
-    # edge rows: slot 1 repeats slot 0 (the oracle gets -1 there), or no block at all
+    # edge rows: slot 1 repeats slot 0 (the block counts once), or no block at all
     rng = np.random.default_rng(7)
     idx_e = idx.cpu().numpy().copy()
-    ref_e = idx_e.copy()
     rows = rng.choice(len(idx_e), 300, replace=False)
     dup, empty = rows[:200], rows[200:]
     for r in dup:
         g = int(rng.integers(w.hkv))
         if idx_e[r, g, 1] >= 0:
             idx_e[r, g, 1] = idx_e[r, g, 0]
-            ref_e[r, g, 1] = -1
     idx_e[empty] = -1
-    ref_e[empty] = -1
+    ref_e = idx_e
     out_e, lse_e = msa.sparse_attn_prefill(cache, q, torch.from_numpy(idx_e).to(DEV), cu_q=cu,
                                            max_rows_per_seq=max(n))
     torch.cuda.synchronize()
@@ -260,12 +258,23 @@ def test_rows_without_blocks(name, over):
     idx2 = idx.clone()
     idx2[empty] = -1
     out, lse = msa.sparse_attn_prefill(cache, q, idx2, cu_q=cu, max_rows_per_seq=T)
+    # a block repeated in the adjacent slot counts once: same as -1 in that slot
+    dup = torch.arange(200, T, 11, device=DEV)
+    dup = dup[(idx[dup, :, 1] >= 0).all(-1)]
+    idx3, idx4 = idx.clone(), idx.clone()
+    idx3[dup, :, 1] = idx3[dup, :, 0]
+    idx4[dup, :, 1] = -1
+    out3, _ = msa.sparse_attn_prefill(cache, q, idx3, cu_q=cu, max_rows_per_seq=T)
+    out4, _ = msa.sparse_attn_prefill(cache, q, idx4, cu_q=cu, max_rows_per_seq=T)
     torch.cuda.synchronize()
     assert cache.device_status() == 0
     assert torch.all(out[empty] == 0) and torch.all(torch.isneginf(lse[empty]))
     keep = torch.ones(T, dtype=torch.bool, device=DEV)
     keep[empty] = False
     assert torch.equal(out[keep].view(torch.int16), ref[keep].view(torch.int16))
+    assert len(dup) > 10
+    assert (out3[dup].float() - out4[dup].float()).abs().max().item() < 1e-6
+    assert not torch.equal(out3[dup], ref[dup])   # the lists did change
 
 
 # ---------------------------------------------------------------------------
@@ -280,6 +289,33 @@ DECODE_CASES = [
     ("topk2", lambda: workloads.paged_decode_bf16(batch=2, ctx=(5000, 700), top_k=2,
                                                   planted=(1, 1))),
 ]
+
+
+def test_decode_repeated_and_empty_block_lists():
+    """Split-k decode: an adjacent repeat of a block counts once, a sequence
+    whose list is all -1 gives 0 and lse = -inf."""
+    w = workloads.paged_decode_bf16(batch=3, ctx=(3000, 5000, 4096))
+    p = workloads.paging(w)
+    cache = new_cache(w, p)
+    lens = fill_context(cache, w)
+    append(cache, w, lens, [L + 1 for L in lens])
+    q = workloads.queries_decode(w, 0, DEV)
+    idx, _ = msa.select_topk(cache, q, w.top_k)
+    ref, _ = msa.sparse_attn_decode(cache, q, idx)
+    idx3, idx4 = idx.clone(), idx.clone()
+    for s_ in (1, 9, 17):   # repeats inside and across the split boundaries
+        idx3[0, :, s_] = idx3[0, :, s_ - 1]
+        idx4[0, :, s_] = -1
+    idx3[2] = -1
+    idx4[2] = -1
+    o3, l3 = msa.sparse_attn_decode(cache, q, idx3)
+    o4, l4 = msa.sparse_attn_decode(cache, q, idx4)
+    torch.cuda.synchronize()
+    assert cache.device_status() == 0
+    assert (o3[0].float() - o4[0].float()).abs().max().item() < 1e-6
+    assert not torch.equal(o3[0], ref[0])
+    assert torch.equal(o3[1].view(torch.int16), ref[1].view(torch.int16))
+    assert torch.all(o3[2] == 0) and torch.all(torch.isneginf(l3[2]))
 
 
 @pytest.mark.parametrize("name,make", DECODE_CASES, ids=[c[0] for c in DECODE_CASES])

@@ -250,6 +250,32 @@ def test_permuted_index_order_and_row_subsets():
     assert np.max(np.abs(one["out"][0] - r["out"][L - 1])) < 1e-15
 
 
+def test_repeated_and_empty_block_lists():
+    """The attended tokens are a set: a block listed twice equals the block
+    listed once; a row without any block attends to nothing (O = 0, lse = -inf),
+    and its neighbours are unaffected."""
+    L, B, d, hq, hkv, k = 64, 8, 16, 4, 2, 4
+    Q, K, V = _rand((L, hq, d), 40), _rand((L, hkv, d), 41), _rand((L, hkv, d), 42)
+    pos = np.arange(L)
+    r = oracle.forward(Q, K, V, pos, B, k, 0.25)
+    idx = r["idx"].copy()
+    rows = [t for t in range(L) if idx[t, 0, 1] >= 0][:5]
+    dup, ref = idx.copy(), idx.copy()
+    for t in rows:
+        dup[t, 0, 1] = dup[t, 0, 0]
+        ref[t, 0, 1] = -1
+    Od, ld = oracle.attend(Q, K, V, pos, dup, B, 0.25)
+    Or, lr = oracle.attend(Q, K, V, pos, ref, B, 0.25)
+    assert np.array_equal(Od, Or) and np.array_equal(ld, lr)
+    assert not np.allclose(Od[rows[0]], r["out"][rows[0]])   # the list did change
+    empty = idx.copy()
+    empty[7] = -1
+    Oe, le = oracle.attend(Q, K, V, pos, empty, B, 0.25)
+    assert np.all(Oe[7] == 0.0) and np.all(np.isneginf(le[7]))
+    others = np.arange(L) != 7
+    assert np.array_equal(Oe[others], r["out"][others])
+
+
 def test_tiny_workload_finds_planted_blocks():
     """Generator + oracle: the tiny workload plants two blocks along the last
     query's mean head direction, so that query ranks them first."""
