@@ -128,7 +128,7 @@ __device__ void write_selection(const uint64_t* keys, int n, int own, int top_k,
 // select_rows
 // ---------------------------------------------------------------------------
 template <typename T, int D, int KMAX>
-__global__ void __launch_bounds__(256) select_rows_kernel(
+__global__ void __launch_bounds__(256, KMAX <= 16 ? 3 : 1) select_rows_kernel(
     const T* __restrict__ q, const int32_t* __restrict__ cu_q, const float* __restrict__ centroids,
     const int32_t* __restrict__ page_table, const int32_t* __restrict__ seq_lens, uint32_t* status,
     int hq, int hkv, int B, int num_pages, int max_blocks, int top_k, int32_t* __restrict__ idx,
@@ -139,7 +139,8 @@ __global__ void __launch_bounds__(256) select_rows_kernel(
   float* qbar = reinterpret_cast<float*>(smem_raw);                  // [kRows][D]
   float* cent = qbar + kRows * D;                                     // [kChunk][CP]
   float* sc = cent + kChunk * CP;                                     // [kRows][kChunk]
-  uint64_t* lists = reinterpret_cast<uint64_t*>(sc + kRows * kChunk); // [kRows][SUBS][KMAX]
+  // the merge lists reuse the chunk buffers once every chunk is scored
+  uint64_t* lists = reinterpret_cast<uint64_t*>(cent);                // [kRows][SUBS][KMAX]
   __shared__ int s_page[kChunk];
 
   const int b = blockIdx.y, g = blockIdx.z;
@@ -253,6 +254,7 @@ __global__ void __launch_bounds__(256) select_rows_kernel(
   // A, B: max(A[i], B[N-1-i]) holds the top N as a bitonic sequence, which a
   // half-cleaner network sorts back into descending order.
   uint64_t* my_list = lists + ((size_t)sr * SUBS + ss) * KMAX;
+  __syncthreads();  // the last chunk's scores are read: the lists may overwrite them
 #pragma unroll
   for (int s = 0; s < KMAX; ++s) my_list[s] = top[s];
   __syncthreads();
@@ -831,8 +833,9 @@ __global__ void __launch_bounds__(32) select_decode_pass2(
 static int kmax_for(int top_k) { return top_k - 1 <= 16 ? 16 : (top_k - 1 <= 32 ? 32 : 64); }
 
 static size_t rows_smem(int D, int kmax) {
-  return (size_t)kRows * D * 4 + (size_t)kChunk * (D + 4) * 4 + (size_t)kRows * kChunk * 4 +
-         (size_t)kRows * (256 / kRows) * kmax * 8;
+  const size_t chunk = (size_t)kChunk * (D + 4) * 4 + (size_t)kRows * kChunk * 4;
+  const size_t lists = (size_t)kRows * (256 / kRows) * kmax * 8;
+  return (size_t)kRows * D * 4 + (chunk > lists ? chunk : lists);
 }
 
 template <typename T, int D, int KMAX>
