@@ -43,17 +43,104 @@ constexpr float kLog2e = 1.4426950408889634f;
 }  // namespace
 
 // ---------------------------------------------------------------------------
-// Planning: for each unit of query tiles (tiles_per_unit * TM consecutive
-// tokens), the union of the tokens' selections, ascending, each block with a
-// 32-bit mask: bit (tile * 16 + token-in-tile) is set when that token selected
-// the block.
+// Token order. The query rows of a sequence are taken in windows of kWin rows;
+// per window and KV group the tokens are dealt into the window's tiles (TM
+// tokens each) greedily: a tile starts from the lowest-indexed token not yet
+// placed and grows by the token whose usable blocks add the fewest new blocks
+// to the tile's union (ties: the lower index). Tokens that selected the same
+// blocks then share a tile, so the union a tile walks shrinks (on the prefill
+// workload from 64 to 54 blocks per 16-token tile). perm[window][g][p] is the
+// window offset of the p-th token of the new order; the attention is the same
+// for any order, only the work changes.
+// ---------------------------------------------------------------------------
+constexpr int kWin = 128;
+
+constexpr int kClusterK = 16;  // block lists of up to 16 entries are clustered (in registers)
+
+// one CTA per region (window, group), a thread per token
+__global__ void __launch_bounds__(kWin) prefill_cluster_kernel(
+    const int32_t* __restrict__ cu_q, const int32_t* __restrict__ seq_lens,
+    const int32_t* __restrict__ block_idx, int hkv, int B, int max_blocks, int top_k, int TM,
+    int wps, uint8_t* __restrict__ perm) {
+  extern __shared__ uint32_t cur[];  // union bitmap of the tile being built
+  __shared__ unsigned s_red[kWin / 32];
+  __shared__ int s_best;
+  const int region = blockIdx.x;
+  const int g = region % hkv;
+  const int w = (region / hkv) % wps;
+  const int b = region / (hkv * wps);
+  const int tid = threadIdx.x;
+  const int row0 = cu_q[b];
+  const int n_rows = cu_q[b + 1] - row0;
+  const int r_lo = w * kWin;
+  if (r_lo >= n_rows) return;
+  const int nw = min(kWin, n_rows - r_lo);
+  uint8_t* pw = perm + (size_t)region * kWin;
+  const int L = seq_lens[b];
+  if (n_rows > L || L > max_blocks * B || top_k > kClusterK) {  // identity order
+    if (tid < nw) pw[tid] = (uint8_t)tid;
+    return;
+  }
+  const int t0 = L - n_rows + r_lo;
+  int my[kClusterK];
+#pragma unroll
+  for (int s = 0; s < kClusterK; ++s) {
+    int j = -1;
+    if (tid < nw && s < top_k) {
+      j = block_idx[((size_t)(row0 + r_lo + tid) * hkv + g) * top_k + s];
+      if (j > (t0 + tid) / B) j = -1;
+    }
+    my[s] = j;
+  }
+  const int rw = ((t0 + nw - 1) / B + 1 + 31) / 32;  // bitmap words of blocks 0 .. last own block
+  bool placed = tid >= nw;
+  for (int p = 0; p < nw; ++p) {
+    const bool seed = (p % TM) == 0;
+    if (seed) {
+      for (int i = tid; i < rw; i += kWin) cur[i] = 0u;
+      __syncthreads();
+    }
+    unsigned key = 0xffffffffu;
+    if (!placed) {
+      unsigned grow = 0;
+      if (!seed) {
+#pragma unroll
+        for (int s = 0; s < kClusterK; ++s)
+          if (my[s] >= 0) grow += ((cur[my[s] >> 5] >> (my[s] & 31)) & 1u) ^ 1u;
+      }
+      key = (grow << 8) | (unsigned)tid;
+    }
+    key = __reduce_min_sync(0xffffffffu, key);
+    if ((tid & 31) == 0) s_red[tid >> 5] = key;
+    __syncthreads();
+    if (tid == 0) {
+      unsigned m = s_red[0];
+      for (int k = 1; k < kWin / 32; ++k) m = min(m, s_red[k]);
+      s_best = (int)(m & 0xffu);
+      pw[p] = (uint8_t)(m & 0xffu);
+    }
+    __syncthreads();
+    if (tid == s_best) {
+      placed = true;
+#pragma unroll
+      for (int s = 0; s < kClusterK; ++s)
+        if (my[s] >= 0) atomicOr(&cur[my[s] >> 5], 1u << (my[s] & 31));
+    }
+    __syncthreads();
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Planning: for each query tile (TM tokens in the window order above), the
+// union of the tokens' selections, ascending, each block with a 32-bit mask:
+// bit i is set when the tile's token i selected the block.
 // ---------------------------------------------------------------------------
 constexpr int kPlanWindow = 4096;
 
 __global__ void __launch_bounds__(128) prefill_plan_kernel(
     const int32_t* __restrict__ cu_q, const int32_t* __restrict__ seq_lens,
     const int32_t* __restrict__ block_idx, uint32_t* status, int hkv, int B, int max_blocks,
-    int top_k, int TM, int tiles_per_unit, int units_per_seq, int ecap,
+    int top_k, int TM, int units_per_seq, int wps, const uint8_t* __restrict__ perm, int ecap,
     int2* __restrict__ entries, int* __restrict__ counts) {
   __shared__ uint32_t bm[kPlanWindow];
   __shared__ int warp_tot[4];
@@ -65,12 +152,16 @@ __global__ void __launch_bounds__(128) prefill_plan_kernel(
   const int tid = threadIdx.x, lane = tid % 32, warp = tid / 32;
   const int row0 = cu_q[b];
   const int n_rows = cu_q[b + 1] - row0;
-  const int r_lo = tt * tiles_per_unit * TM;
+  const int r_lo = tt * TM;
   if (r_lo >= n_rows) {
     if (tid == 0) counts[tile] = 0;
     return;
   }
-  const int nr = min(tiles_per_unit * TM, n_rows - r_lo);
+  const int w = r_lo / kWin;                      // window, and the tile's first order position
+  const int p0 = r_lo % kWin;
+  const int nw = min(kWin, n_rows - w * kWin);
+  const int nr = min(TM, nw - p0);
+  const uint8_t* pw = perm + ((size_t)(b * wps + w) * hkv + g) * kWin;
   const int L = seq_lens[b];
   if (n_rows > L || L > max_blocks * B) {
     if (tid == 0) {
@@ -79,8 +170,8 @@ __global__ void __launch_bounds__(128) prefill_plan_kernel(
     }
     return;
   }
-  const int t_first = L - n_rows + r_lo;
-  const int own_max = (t_first + nr - 1) / B;
+  const int t_win = L - n_rows + w * kWin;       // position of the window's first row
+  const int own_max = (t_win + nw - 1) / B;
   const int R = own_max + 1;
   int2* out = entries + (size_t)tile * ecap;
   if (tid == 0) s_base = 0;
@@ -90,14 +181,15 @@ __global__ void __launch_bounds__(128) prefill_plan_kernel(
     __syncthreads();
     for (int it = tid; it < nr * top_k; it += 128) {
       const int i = it / top_k, s = it % top_k;
-      const int j = block_idx[((size_t)(row0 + r_lo + i) * hkv + g) * top_k + s];
+      const int o = pw[p0 + i];                     // the token's offset in its window
+      const int j = block_idx[((size_t)(row0 + w * kWin + o) * hkv + g) * top_k + s];
       if (j < 0) continue;
-      const int own_i = (t_first + i) / B;
+      const int own_i = (t_win + o) / B;
       if (j > own_i) {
         report(status, MSA_DEV_BAD_INDEX);
         continue;
       }
-      if (j >= w0 && j < w0 + W) atomicOr(&bm[j - w0], 1u << ((i / TM) * 16 + i % TM));
+      if (j >= w0 && j < w0 + W) atomicOr(&bm[j - w0], 1u << i);
     }
     __syncthreads();
     // compaction: thread tid scans words [tid*per, (tid+1)*per)
@@ -213,7 +305,8 @@ __global__ void __launch_bounds__(192, 1) prefill_tc_kernel(
     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
     const bf16* __restrict__ q, const int32_t* __restrict__ cu_q,
     const int32_t* __restrict__ page_table, const int32_t* __restrict__ seq_lens, uint32_t* status,
-    int hq, int hkv, int num_pages, int max_blocks, int units_per_seq, int ecap,
+    int hq, int hkv, int num_pages, int max_blocks, int units_per_seq, int wps,
+    const uint8_t* __restrict__ perm, int ecap,
     const int2* __restrict__ entries, const int* __restrict__ counts, float scale_log2,
     bf16* __restrict__ out, float* __restrict__ lse, gate_t gate) {
   constexpr int TM = 128 / G;              // tokens per query tile (128 rows)
@@ -241,14 +334,32 @@ __global__ void __launch_bounds__(192, 1) prefill_tc_kernel(
   const int pu = (unit / hkv) % units_per_seq;
   const int b = unit / (hkv * units_per_seq);
   const int n_e = counts[unit];
-  if (n_e == 0) return;  // nothing to do (ragged batch) - uniform exit before any sync
   const int2* ent = entries + (size_t)unit * ecap;
   const int row0 = cu_q[b];
   const int n_rows = cu_q[b + 1] - row0;
   const int r_lo = pu * TM;
-  const int nr = min(TM, n_rows - r_lo);
+  const int wdw = r_lo / kWin;                    // window of the tile, and its first order position
+  const int p0 = r_lo % kWin;
+  const int nw = min(kWin, n_rows - wdw * kWin);
+  const int nr = min(TM, nw - p0);
+  const uint8_t* pw = perm + ((size_t)(b * wps + wdw) * hkv + g) * kWin;
   const int L = seq_lens[b];
-  const int t_first = L - n_rows + r_lo;
+  const int t_win = L - n_rows + wdw * kWin;      // position of the window's first row
+  const int row_win = row0 + wdw * kWin;          // global row of the window's first row
+  if (n_e == 0) {
+    // no token of the tile took a block (or the tile lies past the sequence's
+    // rows): its rows attend to nothing, A = 0. Uniform exit before any sync.
+    if (threadIdx.x >= 64) {
+      const int r = threadIdx.x - 64, ti = r / G, h = r % G;
+      if (ti < nr) {
+        const size_t head = ((size_t)row_win + pw[p0 + ti]) * hq + (size_t)g * G + h;
+        for (int c = 0; c < kD; ++c)
+          out[head * kD + c] = __float2bfloat16_rn(gate_apply<bf16>(gate, head, c, kD, 0.f));
+        if (lse) lse[head] = -INFINITY;
+      }
+    }
+    return;
+  }
 
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   if (tid == 0) {
@@ -360,12 +471,14 @@ __global__ void __launch_bounds__(192, 1) prefill_tc_kernel(
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
     const int ti = r / G, h = r % G;               // token within the tile, head in the group
     const bool row_ok = ti < nr;
-    const int t = t_first + ti;                    // position of this row's token
+    const int o_tok = row_ok ? pw[p0 + ti] : 0;    // the token's offset in its window
+    const int t = t_win + o_tok;                   // position of this row's token
+    const size_t qrow = (size_t)row_win + o_tok;   // its global query row
     // Q row -> TMEM (bf16 pairs as 32-bit columns)
     {
       uint32_t qv[32];
       const uint4* src = reinterpret_cast<const uint4*>(
-          q + ((size_t)(row0 + r_lo + ti) * hq + (size_t)g * G + h) * kD);
+          q + (qrow * hq + (size_t)g * G + h) * kD);
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
 #pragma unroll
@@ -405,7 +518,7 @@ __global__ void __launch_bounds__(192, 1) prefill_tc_kernel(
     for (int hv = 0; hv < 2; ++hv) {
       ti_half[hv] = (quarter * 32 + hv * 16 + (lane & 15)) / G;
       ok_half[hv] = ti_half[hv] < nr;
-      t_half[hv] = t_first + ti_half[hv];
+      t_half[hv] = t_win + (ok_half[hv] ? pw[p0 + ti_half[hv]] : 0);
     }
     const bool upper = lane >= 16;  // which 64 columns of the half-mode row
     int2 en_next = ent[0];
@@ -560,7 +673,7 @@ __global__ void __launch_bounds__(192, 1) prefill_tc_kernel(
       // a row that took no block (its token selected none) has an empty sum: A = 0
       const float l = (m_ref == -INFINITY) ? 0.f : l_run;
       const float inv = (l > 0.f) ? 1.f / l : 0.f;
-      const size_t head = (size_t)(row0 + r_lo + ti) * hq + (size_t)g * G + h;
+      const size_t head = qrow * hq + (size_t)g * G + h;
       uint4* dst = reinterpret_cast<uint4*>(out + head * kD);
 #pragma unroll
       for (int c = 0; c < kD / 32; ++c) {
@@ -594,7 +707,7 @@ __global__ void __launch_bounds__(192, 1) prefill_tc_kernel(
         }
       }
       if (row_ok && lse)
-        lse[(size_t)(row0 + r_lo + ti) * hq + (size_t)g * G + h] =
+        lse[qrow * hq + (size_t)g * G + h] =
             (l > 0.f) ? (m_ref + log2f(l)) * 0.6931471805599453f : -INFINITY;
     } else if (go) {
       report(status, MSA_DEV_TIMEOUT);
@@ -619,12 +732,16 @@ static int plan_units(const msa_paged_kv_t* kv, int max_rows, int* ups) {
   return kv->batch * (*ups) * kv->num_kv_heads;
 }
 
+static int windows_per_seq(int max_rows) { return (max_rows + kWin - 1) / kWin; }
+
+// workspace: entries [units][ecap] int2 | counts [units] int | perm [batch][wps][hkv][kWin] u8
 size_t prefill_ws(const msa_paged_kv_t* kv, int max_rows, int top_k) {
   int ups;
   const size_t units = plan_units(kv, max_rows, &ups);
   const int TM = 128 / (kv->num_q_heads / kv->num_kv_heads);
   const size_t ecap = (size_t)TM * top_k;
-  return units * ecap * sizeof(int2) + units * sizeof(int) + 256;
+  const size_t perm = (size_t)kv->batch * windows_per_seq(max_rows) * kv->num_kv_heads * kWin;
+  return units * ecap * sizeof(int2) + units * sizeof(int) + perm + 256;
 }
 
 bool prefill_tc_supported(const msa_paged_kv_t* kv) {
@@ -635,9 +752,9 @@ bool prefill_tc_supported(const msa_paged_kv_t* kv) {
 
 template <int B, int G>
 static cudaError_t launch_tc(const msa_paged_kv_t* kv, const CUtensorMap& tk, const CUtensorMap& tv,
-                             const void* q, const int32_t* cu_q, int units, int ups, int ecap,
-                             const int2* entries, const int* counts, float sl2, void* out,
-                             float* lse, gate_t gate, cudaStream_t st) {
+                             const void* q, const int32_t* cu_q, int units, int ups, int wps,
+                             const uint8_t* perm, int ecap, const int2* entries, const int* counts,
+                             float sl2, void* out, float* lse, gate_t gate, cudaStream_t st) {
   constexpr int NST = (B == 128) ? 3 : 4;
   const size_t smem = (size_t)NST * 2 * B * kD * 2 + 1024;
   auto kern = prefill_tc_kernel<B, G>;
@@ -645,7 +762,7 @@ static cudaError_t launch_tc(const msa_paged_kv_t* kv, const CUtensorMap& tk, co
   if (e != cudaSuccess) return e;
   kern<<<units, 192, smem, st>>>(tk, tv, (const bf16*)q, cu_q, kv->page_table, kv->seq_lens,
                                  kv->status_word, kv->num_q_heads, kv->num_kv_heads, kv->num_pages,
-                                 kv->max_blocks_per_seq, ups, ecap, entries, counts, sl2,
+                                 kv->max_blocks_per_seq, ups, wps, perm, ecap, entries, counts, sl2,
                                  (bf16*)out, lse, gate);
   return cudaGetLastError();
 }
@@ -657,25 +774,33 @@ cudaError_t prefill_tc(const msa_paged_kv_t* kv, const void* q, const int32_t* c
   const int TM = 128 / G;
   int ups;
   const int units = plan_units(kv, max_rows, &ups);
+  const int wps = windows_per_seq(max_rows);
   const int ecap = TM * top_k;
   int2* entries = (int2*)ws;
   int* counts = (int*)(entries + (size_t)units * ecap);
-  prefill_plan_kernel<<<units, 128, 0, st>>>(cu_q, kv->seq_lens, idx, kv->status_word,
-                                             kv->num_kv_heads, B, kv->max_blocks_per_seq, top_k,
-                                             TM, 1, ups, ecap, entries, counts);
-  cudaError_t e = cudaGetLastError();
+  uint8_t* perm = (uint8_t*)(counts + units);
+  const int hkv = kv->num_kv_heads, mb = kv->max_blocks_per_seq;
+  const size_t cl_smem = ((size_t)(mb + 31) / 32) * 4;
+  cudaError_t e = cudaFuncSetAttribute(prefill_cluster_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)cl_smem);
   if (e != cudaSuccess) return e;
+  prefill_cluster_kernel<<<kv->batch * wps * hkv, kWin, cl_smem, st>>>(
+      cu_q, kv->seq_lens, idx, hkv, B, mb, top_k, TM, wps, perm);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  prefill_plan_kernel<<<units, 128, 0, st>>>(cu_q, kv->seq_lens, idx, kv->status_word, hkv, B, mb,
+                                             top_k, TM, ups, wps, perm, ecap, entries, counts);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
   CUtensorMap tk, tv;
-  const uint64_t rows = (uint64_t)kv->num_pages * kv->num_kv_heads * B;
+  const uint64_t rows = (uint64_t)kv->num_pages * hkv * B;
   if (!make_tmap_bf16_2d(&tk, kv->k_pages, rows, kD, 64, B) ||
       !make_tmap_bf16_2d(&tv, kv->v_pages, rows, kD, 64, B))
     return cudaErrorInvalidValue;
   const float sl2 = scale * kLog2e;
   if (B == 128)
-    return G == 8 ? launch_tc<128, 8>(kv, tk, tv, q, cu_q, units, ups, ecap, entries, counts, sl2, out, lse, gate, st)
-                  : launch_tc<128, 16>(kv, tk, tv, q, cu_q, units, ups, ecap, entries, counts, sl2, out, lse, gate, st);
-  return G == 8 ? launch_tc<64, 8>(kv, tk, tv, q, cu_q, units, ups, ecap, entries, counts, sl2, out, lse, gate, st)
-                : launch_tc<64, 16>(kv, tk, tv, q, cu_q, units, ups, ecap, entries, counts, sl2, out, lse, gate, st);
+    return G == 8 ? launch_tc<128, 8>(kv, tk, tv, q, cu_q, units, ups, wps, perm, ecap, entries, counts, sl2, out, lse, gate, st)
+                  : launch_tc<128, 16>(kv, tk, tv, q, cu_q, units, ups, wps, perm, ecap, entries, counts, sl2, out, lse, gate, st);
+  return G == 8 ? launch_tc<64, 8>(kv, tk, tv, q, cu_q, units, ups, wps, perm, ecap, entries, counts, sl2, out, lse, gate, st)
+                : launch_tc<64, 16>(kv, tk, tv, q, cu_q, units, ups, wps, perm, ecap, entries, counts, sl2, out, lse, gate, st);
 }
 
 }  // namespace msa
