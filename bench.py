@@ -528,9 +528,7 @@ def main():
                     "d2h_bytes_per_step": r["d2h"]},
             "gpu_launches": r["launches_per_step"] * args.steps,
             "clocks": r["clocks"],
-            "config": {"workload": w.name, "batch": w.batch, "seq_len": T, "q_heads": w.hq,
-                       "kv_heads": w.hkv, "head_dim": w.d, "block": w.block, "top_k": w.top_k,
-                       "l2": "inputs 0.7 GB per step > 126 MB L2, no flush"},
+            "config": workload_config(w),
         })
         if not args.no_decode and world == 1:
             wd = workloads.paged_decode_bf16()
@@ -566,7 +564,7 @@ def decode_call_bytes(w, step=0):
 
 
 def decode_block(w, args, world, pk):
-    flush = w.name == "decode_1m_bf16"
+    flush = decode_flush(w)
     r = run_decode(w, args.steps, args.warmup, world, flush)
     ms = max_over_ranks(r["step_ms"], world)
     nbytes = decode_bytes(w)
@@ -608,9 +606,25 @@ def decode_main(w, args, world, pk):
     return {"metric": METRIC, "value": d["value"], "unit": "tokens/s", "ms_per_step": d["ms_per_step"],
             "roofline": d["roofline"], "kernels_ms": d["kernels_ms"], "e2e": d["e2e"],
             "clocks": d["clocks"], "gpu_launches": d["gpu_launches"],
-            "config": {"workload": w.name, "batch": w.batch, "q_heads": w.hq, "kv_heads": w.hkv,
-                       "head_dim": w.d, "block": w.block, "top_k": w.top_k,
-                       "context_mean": float(np.mean(w.ctx)), "l2": d["l2"]}}
+            "config": workload_config(w)}
+
+
+def decode_flush(w):
+    """The 1M-context step reads ~41 MB, inside L2: flush it between steps."""
+    return w.name == "decode_1m_bf16"
+
+
+def workload_config(w):
+    """The config object of the JSON line (the same for both arms)."""
+    c = {"workload": w.name, "batch": w.batch, "q_heads": w.hq, "kv_heads": w.hkv,
+         "head_dim": w.d, "block": w.block, "top_k": w.top_k}
+    if w.kind == "prefill":
+        c.update({"seq_len": w.ctx[0], "l2": "inputs 0.7 GB per step > 126 MB L2, no flush"})
+    else:
+        c.update({"context_mean": float(np.mean(w.ctx)),
+                  "l2": ("256 MB write between steps" if decode_flush(w)
+                         else "step reads > 126 MB L2, no flush")})
+    return c
 
 
 def cpu_baseline(w, args):
@@ -645,7 +659,7 @@ def reference_arm(w, args):
             "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * secs / len(steps), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": w.name},
+            "config": workload_config(w),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": thr, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
