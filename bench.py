@@ -254,14 +254,14 @@ def run_prefill(w, steps, warmup, world):
     k_ms = [time_graph(gg, steps) for gg in g_ops]
     total_ms = step_ms * steps
 
-    # executed (union) tile-blocks of the tensor-core schedule, for context
+    # executed (union) tile-blocks of the tensor-core schedule, for context: the
+    # plan's per-tile union sizes, read back from the call's workspace (entries
+    # [units][ecap] int2, then counts [units] int32)
     G = w.group
     TM = 128 // G
-    sel = idx.cpu().numpy()
-    union_blocks = 0
-    for g in range(w.hkv):
-        for t0_ in range(0, T, TM):
-            union_blocks += len(np.unique(sel[t0_:t0_ + TM, g][sel[t0_:t0_ + TM, g] >= 0]))
+    units = ((T + TM - 1) // TM) * w.hkv
+    off = units * TM * w.top_k * 8
+    union_blocks = int(ws_att[off:off + 4 * units].view(torch.int32).sum().item())
 
     # end to end through the C ABI from pinned host buffers
     hq_ = q.cpu().pin_memory()
@@ -299,7 +299,7 @@ def run_prefill(w, steps, warmup, world):
         raise RuntimeError(f"device status {status:#x}")
     return {"total_ms": total_ms, "kernel_ms": k_ms, "clocks": clk.summary(),
             "union_blocks": union_blocks, "e2e_ms": e2e_ms, "h2d": h2d, "d2h": d2h,
-            "launches_per_step": 4}
+            "launches_per_step": 5}
 
 
 # ---------------------------------------------------------------------------
@@ -517,7 +517,7 @@ def main():
                          "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"],
                          "traffic": traffic,
                          "peak_source": f"{pk['source']} bf16 (burst cuBLAS)",
-                         "kernel": "msa_sparse_attn_prefill (plan + prefill_tc_kernel)",
+                         "kernel": "msa_sparse_attn_prefill (cluster + plan + prefill_tc_kernel)",
                          "algorithmic_flops_per_launch": flops,
                          "executed_mma_flops_per_launch": executed,
                          "executed_tflops": executed / (attn_ms * 1e-3) / 1e12},

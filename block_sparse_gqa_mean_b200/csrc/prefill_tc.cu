@@ -64,7 +64,6 @@ __global__ void __launch_bounds__(kWin) prefill_cluster_kernel(
     int wps, uint8_t* __restrict__ perm) {
   extern __shared__ uint32_t cur[];  // union bitmap of the tile being built
   __shared__ unsigned s_red[kWin / 32];
-  __shared__ int s_best;
   const int region = blockIdx.x;
   const int g = region % hkv;
   const int w = (region / hkv) % wps;
@@ -113,14 +112,12 @@ __global__ void __launch_bounds__(kWin) prefill_cluster_kernel(
     key = __reduce_min_sync(0xffffffffu, key);
     if ((tid & 31) == 0) s_red[tid >> 5] = key;
     __syncthreads();
-    if (tid == 0) {
-      unsigned m = s_red[0];
-      for (int k = 1; k < kWin / 32; ++k) m = min(m, s_red[k]);
-      s_best = (int)(m & 0xffu);
-      pw[p] = (uint8_t)(m & 0xffu);
-    }
-    __syncthreads();
-    if (tid == s_best) {
+    unsigned m = s_red[0];  // every thread reads the four warp minima
+#pragma unroll
+    for (int k = 1; k < kWin / 32; ++k) m = min(m, s_red[k]);
+    const int best = (int)(m & 0xffu);
+    if (tid == 0) pw[p] = (uint8_t)best;
+    if (tid == best) {
       placed = true;
 #pragma unroll
       for (int s = 0; s < kClusterK; ++s)
