@@ -28,6 +28,17 @@ Citations (page title, section):
                  Practical Deployment", section 4.3, step 6 of the computation
                  flow: O = Gate * A + (1 - Gate) * X, the gate a scalar or
                  varying with the dimension (X given by the caller).
+  * token_scores, token_select, attend_tokens - the token-granular variant of
+                 "Sparse Attention + Linear Backbones: How LLM Long-Context
+                 Architectures Are Evolving", sections 5.1-5.3 and 5.5: a
+                 lightweight multi-head indexer without positional encoding
+                 scores every historical position, the top-K positions are
+                 kept, and the main attention runs over those positions only.
+                 The page leaves the indexer's form open; the reading here
+                 mirrors the block path: s(t, u) = sum over indexer heads h of
+                 qI[t, h] . kI[u] for u <= t, exp-free, the query's own
+                 position always kept, ties to the lower position (pure numpy,
+                 fp64).
 """
 from __future__ import annotations
 
@@ -185,3 +196,65 @@ def _widen(x):
     if x.dtype == np.uint16:
         return (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
     return x.astype(np.float64)
+
+
+# --------------------------------------------------------------------------
+# token-granular variant (indexer over every position, top-K tokens)
+# --------------------------------------------------------------------------
+def token_scores(QI, KI, pos) -> np.ndarray:
+    """s[r, u] = sum_h QI[r, h] . KI[u] in fp64 for u <= pos[r]; -inf after.
+    QI: [R, Hi, di] indexer queries; KI: [L, di] indexer keys (one per position)."""
+    qi = np.asarray(_widen(QI), dtype=np.float64)
+    ki = np.asarray(_widen(KI), dtype=np.float64)
+    pos = np.asarray(pos, dtype=np.int64)
+    S = np.einsum("rhd,ud->ru", qi, ki)
+    future = np.arange(ki.shape[0])[None, :] > pos[:, None]
+    S[future] = -np.inf
+    return S
+
+
+def token_select(S: np.ndarray, pos, top_k: int):
+    """(idx [R, top_k] int32 ascending, -1 padded; gap [R]) of the kept positions:
+    the own position pos[r] plus the top_k - 1 best earlier positions (scores
+    descending, ties to the lower position). gap = score of the last kept
+    earlier position minus the best dropped one (+inf when nothing is dropped)."""
+    pos = np.asarray(pos, dtype=np.int64)
+    R = S.shape[0]
+    idx = np.full((R, top_k), -1, dtype=np.int32)
+    gap = np.full(R, np.inf)
+    for r in range(R):
+        t = int(pos[r])
+        cand = np.arange(t)                                # earlier positions
+        order = cand[np.lexsort((cand, -S[r, :t]))] if t else cand
+        take = min(top_k - 1, t)
+        kept = np.sort(np.concatenate([order[:take], [t]]))
+        idx[r, :len(kept)] = kept
+        if 0 < take < t:
+            gap[r] = S[r, order[take - 1]] - S[r, order[take]]
+    return idx, gap
+
+
+def attend_tokens(Q, K, V, pos, tok_idx, scale: float):
+    """(O [R, Hq, d], lse [R, Hq]) of exact attention of row r over the listed
+    positions u (tok_idx[r], -1 padding, a repeat counts once, u <= pos[r]),
+    the query head h reading KV head h // (Hq // Hkv)."""
+    q = np.asarray(_widen(Q), dtype=np.float64)
+    k = np.asarray(_widen(K), dtype=np.float64)
+    v = np.asarray(_widen(V), dtype=np.float64)
+    pos = np.asarray(pos, dtype=np.int64)
+    R, hq, d = q.shape
+    hkv = k.shape[1]
+    G = hq // hkv
+    O = np.zeros((R, hq, d))
+    lse = np.full((R, hq), -np.inf)
+    for r in range(R):
+        u = np.unique(tok_idx[r][(tok_idx[r] >= 0) & (tok_idx[r] <= pos[r])])
+        if len(u) == 0:
+            continue
+        for h in range(hq):
+            logit = scale * (k[u, h // G] @ q[r, h])
+            m = logit.max()
+            w = np.exp(logit - m)
+            O[r, h] = (w / w.sum()) @ v[u, h // G]
+            lse[r, h] = m + np.log(w.sum())
+    return O, lse

@@ -319,3 +319,93 @@ def test_gate_widens_bf16_branch():
     A = np.array([[[0.5, 0.25]]])
     out = oracle.gate(A, np.array([[0.25]]), x)
     assert np.array_equal(out, 0.25 * A + 0.75 * np.array([[[1.5, -2.25]]]))
+
+
+# --------------------------------------------------------------------------
+# token-granular variant (indexer over every position, top-K tokens)
+# --------------------------------------------------------------------------
+def test_token_topk_all_positions_is_dense_causal():
+    """K >= L keeps every earlier position: dense causal attention (torch SDPA)."""
+    L, d, hq, hkv, hi, di = 70, 16, 4, 2, 3, 8
+    Q, K, V = _rand((L, hq, d), 50), _rand((L, hkv, d), 51), _rand((L, hkv, d), 52)
+    QI, KI = _rand((L, hi, di), 53), _rand((L, di), 54)
+    pos = np.arange(L)
+    S = oracle.token_scores(QI, KI, pos)
+    idx, gap = oracle.token_select(S, pos, L + 5)
+    for r in range(L):
+        assert list(idx[r, :r + 1]) == list(range(r + 1)) and np.all(idx[r, r + 1:] == -1)
+    assert np.all(np.isinf(gap))
+    O, _ = oracle.attend_tokens(Q, K, V, pos, idx, 0.3)
+    mask = torch.from_numpy(np.tril(np.ones((L, L), dtype=bool)))
+    assert np.max(np.abs(O - _sdpa_ref(Q, K, V, mask, 0.3))) < 1e-12
+
+
+def test_token_topk_one_is_the_own_position():
+    """K = 1 keeps only the query's own position: O = v_t, lse = scale q.k_t."""
+    L, d, hq, hkv = 40, 8, 4, 2
+    Q, K, V = _rand((L, hq, d), 60), _rand((L, hkv, d), 61), _rand((L, hkv, d), 62)
+    pos = np.arange(L)
+    S = oracle.token_scores(_rand((L, 2, 8), 63), _rand((L, 8), 64), pos)
+    idx, _ = oracle.token_select(S, pos, 1)
+    assert np.array_equal(idx[:, 0], pos)
+    O, lse = oracle.attend_tokens(Q, K, V, pos, idx, 0.5)
+    v, q, k = V.double().numpy(), Q.double().numpy(), K.double().numpy()
+    for h in range(hq):
+        assert np.array_equal(O[:, h], v[:, h // 2])
+        assert np.max(np.abs(lse[:, h] - 0.5 * np.einsum("rd,rd->r", q[:, h], k[:, h // 2]))) < 1e-12
+
+
+def test_token_select_brute_force_and_ties():
+    """Every kept earlier position scores at least as high as every dropped one;
+    among equal scores the lower position is kept; the scores are the head sum
+    of dot products and ignore the future."""
+    L, hi, di, K_ = 30, 3, 5, 6
+    QI, KI = _rand((L, hi, di), 70), _rand((L, di), 71)
+    KI[10] = KI[4]                          # exact ties between positions 4 and 10
+    KI[20] = KI[4]
+    pos = np.arange(L)
+    S = oracle.token_scores(QI, KI, pos)
+    q, k = QI.double().numpy(), KI.double().numpy()
+    for r in range(L):
+        for u in range(L):
+            want = -np.inf if u > r else sum(float(q[r, h] @ k[u]) for h in range(hi))
+            assert S[r, u] == want or abs(S[r, u] - want) < 1e-12
+    idx, gap = oracle.token_select(S, pos, K_)
+    for r in range(L):
+        kept = [int(u) for u in idx[r] if u >= 0]
+        assert r in kept and len(kept) == min(K_, r + 1) and kept == sorted(kept)
+        earlier = [u for u in kept if u != r]
+        dropped = [u for u in range(r) if u not in kept]
+        for a in earlier:
+            for b in dropped:
+                assert S[r, a] > S[r, b] or (S[r, a] == S[r, b] and a < b)
+        if dropped and earlier:
+            assert gap[r] == min(S[r, a] for a in earlier) - max(S[r, b] for b in dropped)
+    # rows 21 and 25 have the cut inside the tied group: the lower positions stay
+    for r in (21, 25):
+        kept = set(int(u) for u in idx[r] if u >= 0)
+        assert sorted(t for t in (4, 10, 20) if t in kept) == [4, 10]
+
+
+def test_token_path_equals_block_path_on_constant_blocks():
+    """Keys constant within each block, indexer = the group's query heads over
+    the keys, query rows at block starts: the top (k-1) B earlier tokens are
+    exactly the k-1 best blocks, so token attention (own position + those
+    tokens) equals the block oracle's attention over its own selection."""
+    B, nb, d, hq, hkv, k = 8, 9, 16, 4, 1, 4
+    L = B * nb
+    base = _rand((nb, hkv, d), 80)
+    K = base.repeat_interleave(B, dim=0)               # [L, 1, d], constant per block
+    Q, V = _rand((L, hq, d), 81), _rand((L, hkv, d), 82)
+    pos = np.arange(B * (k - 1), L, B)                   # block starts with >= k-1 past blocks
+    Qr = Q[pos]
+    blk = oracle.forward(Qr, K, V, pos, B, k, 0.25)
+    S = oracle.token_scores(Qr, K[:, 0], pos)
+    idx, _ = oracle.token_select(S, pos, (k - 1) * B + 1)
+    for r, t in enumerate(pos):
+        past = sorted(int(j) for j in blk["idx"][r, 0] if 0 <= j < t // B)
+        want = sorted([u for j in past for u in range(j * B, (j + 1) * B)] + [int(t)])
+        assert [int(u) for u in idx[r] if u >= 0] == want
+    O, lse = oracle.attend_tokens(Qr, K, V, pos, idx, 0.25)
+    assert np.max(np.abs(O - blk["out"])) < 1e-12
+    assert np.max(np.abs(lse - blk["lse"])) < 1e-12
