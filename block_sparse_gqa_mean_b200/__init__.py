@@ -29,13 +29,13 @@ LIB_PATH = os.path.join(_PKG, "libmsa.so")
 
 MSA_OK, MSA_ERR_INVALID_ARG, MSA_ERR_UNSUPPORTED, MSA_ERR_WORKSPACE, MSA_ERR_CUDA = range(5)
 MSA_DTYPE_BF16, MSA_DTYPE_F32 = 0, 1
-MSA_OP_SELECT, MSA_OP_PREFILL, MSA_OP_DECODE = 0, 1, 2
+MSA_OP_SELECT, MSA_OP_PREFILL, MSA_OP_DECODE, MSA_OP_SELECT_TOKENS = 0, 1, 2, 3
 MSA_DEV_BAD_PAGE, MSA_DEV_BAD_LENGTH, MSA_DEV_BAD_INDEX, MSA_DEV_TIMEOUT = 1, 2, 4, 8
 
 EXPORTS = ("msa_build_block_cache", "msa_select_topk", "msa_sparse_attn_prefill",
            "msa_sparse_attn_decode", "msa_sparse_attn_prefill_gated",
            "msa_sparse_attn_decode_gated", "msa_sparse_attn_decode_noalloc", "msa_workspace_size",
-           "msa_status_string", "msa_version")
+           "msa_status_string", "msa_version", "msa_select_tokens", "msa_sparse_attn_decode_tokens")
 
 
 class MsaError(RuntimeError):
@@ -87,6 +87,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                                                   I32, P, P, P, P, SZ, P]
     lib.msa_sparse_attn_decode_gated.argtypes = [KV, P, P, I32, ctypes.c_float, P, I32, P, P, P, P,
                                                  SZ, P]
+    lib.msa_select_tokens.argtypes = [KV, P, P, I32, I32, P, P, SZ, P]
+    lib.msa_sparse_attn_decode_tokens.argtypes = [KV, P, P, I32, ctypes.c_float, P, P, P]
     lib.msa_workspace_size.argtypes = [ctypes.c_int, KV, I32, I32, I32]
     lib.msa_workspace_size.restype = SZ
     lib.msa_status_string.argtypes = [ctypes.c_int]
@@ -94,7 +96,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.msa_version.restype = I32
     for name in ("msa_build_block_cache", "msa_select_topk", "msa_sparse_attn_prefill",
                  "msa_sparse_attn_decode", "msa_sparse_attn_prefill_gated",
-                 "msa_sparse_attn_decode_gated", "msa_sparse_attn_decode_noalloc"):
+                 "msa_sparse_attn_decode_gated", "msa_sparse_attn_decode_noalloc",
+                 "msa_select_tokens", "msa_sparse_attn_decode_tokens"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -333,6 +336,47 @@ def sparse_attn_decode_noalloc(cache: PagedKVCache, q: torch.Tensor, block_idx: 
     _check(lib.msa_sparse_attn_decode_noalloc(ctypes.byref(kv), _ptr(q), _ptr(block_idx), top_k,
                                               scale, _ptr(out), _ptr(lse), _stream(stream)),
            "msa_sparse_attn_decode_noalloc")
+    return out, lse
+
+
+def select_tokens(cache: PagedKVCache, ki_pages: torch.Tensor, qi: torch.Tensor, top_k: int,
+                  tok_idx: Optional[torch.Tensor] = None,
+                  workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Token-granular selection for one new query per sequence (at seq_lens-1):
+    ki_pages [num_pages, block_size, head_dim] (one indexer key per position,
+    paged with the cache's page table), qi [batch, num_index_heads, head_dim].
+    Returns tok_idx [batch, top_k] int32: the kept positions ascending (the
+    query's own position last), -1 padded."""
+    lib = load_library()
+    _require_cuda(ki_pages, qi, tok_idx)
+    if tok_idx is None:
+        tok_idx = torch.empty(qi.shape[0], top_k, dtype=torch.int32, device=qi.device)
+    ws, ws_bytes = _workspace(MSA_OP_SELECT_TOKENS, cache, qi.shape[0], 1, top_k, workspace)
+    kv = cache.struct()
+    _check(lib.msa_select_tokens(ctypes.byref(kv), _ptr(ki_pages), _ptr(qi), qi.shape[1], top_k,
+                                 _ptr(tok_idx), _ptr(ws), ws_bytes, _stream(stream)),
+           "msa_select_tokens")
+    return tok_idx
+
+
+def sparse_attn_decode_tokens(cache: PagedKVCache, q: torch.Tensor, tok_idx: torch.Tensor,
+                              softmax_scale: Optional[float] = None,
+                              out: Optional[torch.Tensor] = None,
+                              lse: Optional[torch.Tensor] = None, want_lse: bool = True,
+                              stream=None):
+    """Attention of one new query per sequence over the positions in tok_idx."""
+    lib = load_library()
+    _require_cuda(q, tok_idx, out, lse)
+    top_k = tok_idx.shape[-1]
+    scale = 1.0 / math.sqrt(cache.head_dim) if softmax_scale is None else softmax_scale
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty(q.shape[0], q.shape[1], dtype=torch.float32, device=q.device)
+    kv = cache.struct()
+    _check(lib.msa_sparse_attn_decode_tokens(ctypes.byref(kv), _ptr(q), _ptr(tok_idx), top_k,
+                                             scale, _ptr(out), _ptr(lse), _stream(stream)),
+           "msa_sparse_attn_decode_tokens")
     return out, lse
 
 

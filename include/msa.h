@@ -100,7 +100,8 @@ typedef struct msa_paged_kv {
 typedef enum msa_op {
   MSA_OP_SELECT = 0,
   MSA_OP_PREFILL = 1,
-  MSA_OP_DECODE = 2
+  MSA_OP_DECODE = 2,
+  MSA_OP_SELECT_TOKENS = 3
 } msa_op_t;
 
 /*
@@ -279,6 +280,46 @@ msa_status_t msa_sparse_attn_decode_noalloc(const msa_paged_kv_t* kv, const void
                                             const int32_t* block_idx, int32_t top_k,
                                             float softmax_scale, void* out, float* lse,
                                             msa_stream_t stream);
+
+/*
+ * msa_select_tokens / msa_sparse_attn_decode_tokens - the token-granular
+ * variant for one new query per sequence (decode): a lightweight indexer
+ * scores every earlier position and the attention runs over the kept
+ * positions only.
+ *
+ * Follows "Sparse Attention + Linear Backbones: How LLM Long-Context
+ * Architectures Are Evolving", sections 5.1-5.3 and 5.5 (an indexer without
+ * positional encoding scores every historical position; top-K positions are
+ * kept; attention over those positions). The page leaves the indexer's form
+ * open; it is read here like the block score: for the query at t = seq_lens[b]-1
+ *   s(u) = sum_h qi[b][h] . ki[u]        (u < t; fp32: the heads summed left to
+ *                                         right, then one fma chain in
+ *                                         coordinate order),
+ *   kept = {t} plus the top_k-1 best u < t (all of them when t < top_k),
+ *          ties to the lower position.
+ *
+ *   ki_pages          : device [num_pages][block_size][head_dim], kv->dtype:
+ *                       one indexer key per position, paged with kv's page
+ *                       table (written by the caller).
+ *   qi                : device [batch][num_index_heads][head_dim], kv->dtype.
+ *   tok_idx           : device out [batch][top_k] int32, the kept positions
+ *                       ascending (t last), -1 padded.
+ *   workspace         : device scratch, msa_workspace_size(MSA_OP_SELECT_TOKENS,
+ *                       kv, batch, 1, top_k) bytes (one fp32 score per position).
+ *
+ * msa_sparse_attn_decode_tokens: out / lse as for msa_sparse_attn_decode, over
+ * the positions listed in tok_idx[b] (shared by all KV groups; -1 padding, a
+ * position repeated in the adjacent slot counts once, a row without any
+ * position gives 0 and lse = -inf).
+ */
+msa_status_t msa_select_tokens(const msa_paged_kv_t* kv, const void* ki_pages, const void* qi,
+                               int32_t num_index_heads, int32_t top_k, int32_t* tok_idx,
+                               void* workspace, size_t workspace_bytes, msa_stream_t stream);
+
+msa_status_t msa_sparse_attn_decode_tokens(const msa_paged_kv_t* kv, const void* q,
+                                           const int32_t* tok_idx, int32_t top_k,
+                                           float softmax_scale, void* out, float* lse,
+                                           msa_stream_t stream);
 
 /* Scratch bytes that `op` needs for these sizes (num_rows / max_rows_per_seq
  * as passed to the op; batch and 1 for decode). 0 means no scratch. */

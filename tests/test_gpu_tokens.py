@@ -1,0 +1,105 @@
+"""Token-granular variant (decode): indexer selection and attention over the
+kept positions against the oracle.
+
+"Sparse Attention + Linear Backbones: How LLM Long-Context Architectures Are
+Evolving", sections 5.1-5.5: an indexer scores every earlier position, the
+top-K positions are kept, and attention runs over those only. Selection is
+bit-exact where the oracle's gap between the last kept and the best dropped
+earlier position is at least 1e-2; elsewhere the kept set must score within
+1e-3 of the oracle's cut. Attention is checked on the oracle's own positions.
+"""
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_gqa_mean_b200 as msa
+import oracle
+import workloads
+from msa_harness import GAP_MIN, append, compare, fill_context, new_cache
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+HI = 8
+
+
+def _index_pages(w, p, lens):
+    """Indexer keys of every sequence written into pages of the cache's page table."""
+    ki = torch.zeros(p.num_pages, w.block, w.d, dtype=w.torch_dtype, device=DEV)
+    for b in range(w.batch):
+        L = lens[b]
+        KI = workloads.indexer_keys(w, b, 0, L, DEV)
+        for j in range((L + w.block - 1) // w.block):
+            rows = min(w.block, L - j * w.block)
+            ki[int(p.table[b, j]), :rows] = KI[j * w.block:j * w.block + rows]
+    return ki
+
+
+@pytest.mark.parametrize("top_k", [1, 256, 6000])
+def test_token_decode_selection_and_attention(top_k):
+    w = workloads.paged_decode_bf16(batch=3, ctx=(3000, 5000, 4096))
+    p = workloads.paging(w)
+    cache = new_cache(w, p)
+    lens = fill_context(cache, w)
+    after = [L + 1 for L in lens]
+    append(cache, w, lens, after)
+    ki = _index_pages(w, p, after)
+    qi = workloads.indexer_queries(w, 0, HI, DEV)
+    q = workloads.queries_decode(w, 0, DEV)
+    idx = msa.select_tokens(cache, ki, qi, top_k)
+    torch.cuda.synchronize()
+    assert cache.device_status() == 0
+    gi = idx.cpu().numpy()
+    oidx_all, refs = [], []
+    found = [0, 0]
+    for b in range(w.batch):
+        L = after[b]
+        pos = np.array([L - 1])
+        KI = workloads.indexer_keys(w, b, 0, L)
+        S = oracle.token_scores(qi[b:b + 1].cpu(), KI, pos)
+        oidx, gap = oracle.token_select(S, pos, top_k)
+        row = gi[b]
+        kept = [int(u) for u in row if u >= 0]
+        assert kept == sorted(set(kept)) and kept[-1] == L - 1
+        assert len(kept) == min(top_k, L) and np.all(row[len(kept):] == -1)
+        if gap[0] >= GAP_MIN:
+            assert np.array_equal(row, oidx[0])
+        elif not np.array_equal(row, oidx[0]):
+            earlier = [u for u in kept if u != L - 1]
+            cut = np.sort(S[0, :L - 1])[::-1][len(earlier) - 1]
+            assert all(S[0, u] >= cut - 1e-3 for u in earlier)
+        pt = [u for u in workloads.planted_tokens(w, b) if u < L - 1]
+        found[0] += len(set(pt) & set(kept))
+        found[1] += len(pt)
+        K, V = workloads.keys(w, b, 0, L), workloads.values(w, b, 0, L)
+        O, _ = oracle.attend_tokens(q[b:b + 1].cpu(), K, V, pos, oidx, w.softmax_scale)
+        oidx_all.append(oidx)
+        refs.append(O)
+    if top_k == 256:
+        assert found[0] >= 0.75 * found[1], found
+    oi = torch.from_numpy(np.concatenate(oidx_all)).to(DEV)
+    out, lse = msa.sparse_attn_decode_tokens(cache, q, oi)
+    torch.cuda.synchronize()
+    assert cache.device_status() == 0
+    compare(out, np.concatenate(refs), w.dtype)
+
+
+def test_token_decode_repeated_and_empty_lists():
+    w = workloads.paged_decode_bf16(batch=2, ctx=(2000, 2500))
+    p = workloads.paging(w)
+    cache = new_cache(w, p)
+    lens = fill_context(cache, w)
+    after = [L + 1 for L in lens]
+    append(cache, w, lens, after)
+    q = workloads.queries_decode(w, 0, DEV)
+    base = torch.arange(0, 2000, 7, dtype=torch.int32)[:200]
+    idx = torch.stack([base, base]).to(DEV)
+    idx3, idx4 = idx.clone(), idx.clone()
+    idx3[0, 1::2] = idx3[0, 0::2]        # every odd slot repeats its neighbour
+    idx4[0, 1::2] = -1
+    idx3[1] = -1
+    o3, l3 = msa.sparse_attn_decode_tokens(cache, q, idx3)
+    o4, _ = msa.sparse_attn_decode_tokens(cache, q, idx4)
+    torch.cuda.synchronize()
+    assert cache.device_status() == 0
+    assert (o3[0].float() - o4[0].float()).abs().max().item() < 1e-6
+    assert torch.all(o3[1] == 0) and torch.all(torch.isneginf(l3[1]))

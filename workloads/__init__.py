@@ -234,6 +234,7 @@ ALL = {
 # small parameters (CPU)
 # --------------------------------------------------------------------------
 _T_Q, _T_K, _T_V, _T_U, _T_PLANT, _T_PERM, _T_QD, _T_TINY = range(1, 9)
+_T_KI, _T_QI, _T_PTOK, _T_UI = range(9, 13)  # token-granular indexer inputs
 
 
 @lru_cache(maxsize=64)
@@ -351,6 +352,47 @@ def new_tokens(w: Workload, step: int, device="cpu", seqs=None):
         ks.append(keys(w, b, p, p + 1, device))
         vs.append(values(w, b, p, p + 1, device))
     return torch.cat(ks, 0), torch.cat(vs, 0)
+
+
+# --------------------------------------------------------------------------
+# token-granular indexer inputs (synthetic: the indexer's weights are not given)
+# --------------------------------------------------------------------------
+@lru_cache(maxsize=64)
+def planted_tokens(w: Workload, b: int, count: int = 32) -> List[int]:
+    """Sorted positions of sequence b whose indexer keys lean toward the
+    sequence's indexer direction (CPU)."""
+    gen = cpu_generator(w.seed, _T_PTOK, b)
+    n = w.total_len(b)
+    return sorted(int(x) for x in torch.randperm(n, generator=gen)[:min(count, n)])
+
+
+def _index_direction(w: Workload, b: int) -> torch.Tensor:
+    z = gauss((w.seed, _T_UI, b), 0, w.d, "cpu").to(torch.float64)
+    return (z / z.norm()).to(torch.float32)
+
+
+def indexer_keys(w: Workload, b: int, u0: int, u1: int, device="cpu",
+                 delta: float = 16.0) -> torch.Tensor:
+    """Indexer keys of sequence b at positions [u0, u1): [n, d] in w's dtype,
+    N(0, 1) plus delta along the sequence's indexer direction at the planted
+    positions."""
+    n = u1 - u0
+    z = gauss((w.seed, _T_KI, b), u0 * w.d, n * w.d, device).view(n, w.d)
+    pt = [p - u0 for p in planted_tokens(w, b) if u0 <= p < u1]
+    if pt:
+        z[torch.tensor(pt, device=z.device)] += (_index_direction(w, b) * delta).to(z.device)
+    return z.to(w.torch_dtype)
+
+
+def indexer_queries(w: Workload, step: int, heads: int, device="cpu",
+                    a: float = 2.0) -> torch.Tensor:
+    """Indexer queries of decode step `step`: [batch, heads, d], N(0, 1) plus a
+    along the sequence's indexer direction in every head."""
+    out = []
+    for b in range(w.batch):
+        z = gauss((w.seed, _T_QI, b), step * heads * w.d, heads * w.d, device).view(heads, w.d)
+        out.append(z + (_index_direction(w, b) * a).to(z.device)[None])
+    return torch.stack(out).to(w.torch_dtype)
 
 
 # --------------------------------------------------------------------------
