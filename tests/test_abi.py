@@ -48,3 +48,42 @@ def test_null_cache_is_rejected_without_a_gpu():
     assert lib.msa_select_topk(None, None, None, 1, 1, 4, None, None, None, 0, None) == \
         msa.MSA_ERR_INVALID_ARG
     assert lib.msa_workspace_size(msa.MSA_OP_DECODE, None, 1, 1, 4) == 0
+
+
+def _fake_kv(batch=2, num_pages=64, max_blocks=16, hq=32, hkv=8, d=128, B=64):
+    """A cache descriptor with aligned placeholder pointers: host-side checks
+    only (nothing here reaches a kernel)."""
+    kv = msa._PagedKV()
+    kv.batch, kv.num_pages, kv.max_blocks_per_seq = batch, num_pages, max_blocks
+    kv.num_q_heads, kv.num_kv_heads, kv.head_dim, kv.block_size = hq, hkv, d, B
+    kv.dtype = 0  # bf16
+    for name in ("k_pages", "v_pages", "centroids", "page_table", "seq_lens", "status_word"):
+        setattr(kv, name, 0x10000)
+    return kv
+
+
+def test_token_workspace_and_argument_checks_without_a_gpu():
+    """The token selection's scratch is one fp32 score per cache position of
+    every sequence, whatever top_k (top-K 2048 and beyond is the point of the
+    token variant); bad arguments are refused before any launch."""
+    lib = msa.load_library()
+    kv = _fake_kv()
+    for top_k in (1, 256, 2048, 6000):
+        assert lib.msa_workspace_size(msa.MSA_OP_SELECT_TOKENS, ctypes.byref(kv), 2, 1, top_k) == \
+            2 * 16 * 64 * 4
+    assert lib.msa_workspace_size(msa.MSA_OP_DECODE, ctypes.byref(kv), 2, 1, 300) == 0
+    P = ctypes.c_void_p
+    ok = P(0x20000)
+    # zero indexer heads, a null output, an unaligned query, a short workspace
+    assert lib.msa_select_tokens(ctypes.byref(kv), ok, ok, 0, 16, ok, ok, 1 << 20, None) == \
+        msa.MSA_ERR_INVALID_ARG
+    assert lib.msa_select_tokens(ctypes.byref(kv), ok, ok, 4, 16, None, ok, 1 << 20, None) == \
+        msa.MSA_ERR_INVALID_ARG
+    assert lib.msa_select_tokens(ctypes.byref(kv), ok, P(0x20002), 4, 16, ok, ok, 1 << 20,
+                                 None) == msa.MSA_ERR_INVALID_ARG
+    assert lib.msa_select_tokens(ctypes.byref(kv), ok, ok, 4, 16, ok, ok, 100, None) == \
+        msa.MSA_ERR_WORKSPACE
+    assert lib.msa_sparse_attn_decode_tokens(ctypes.byref(kv), ok, ok, 0, 0.1, ok, None, None) == \
+        msa.MSA_ERR_INVALID_ARG
+    assert lib.msa_sparse_attn_decode_tokens(ctypes.byref(kv), ok, ok, 16, -1.0, ok, None,
+                                             None) == msa.MSA_ERR_INVALID_ARG
