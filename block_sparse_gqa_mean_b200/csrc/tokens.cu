@@ -2,7 +2,7 @@
 //
 // "Sparse Attention + Linear Backbones: How LLM Long-Context Architectures Are
 // Evolving", sections 5.1-5.3 and 5.5: a lightweight multi-head indexer
-// without positional encoding scores every historical position, the top-K
+// without positional encoding rates all earlier positions, the top-K
 // positions are kept, and the main attention runs over those positions only.
 // The indexer's form is not given; it is read here the way the block score is
 // defined: s(t, u) = sum over indexer heads h of qI[h] . kI[u], exp-free,

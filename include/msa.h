@@ -289,7 +289,7 @@ msa_status_t msa_sparse_attn_decode_noalloc(const msa_paged_kv_t* kv, const void
  *
  * Follows "Sparse Attention + Linear Backbones: How LLM Long-Context
  * Architectures Are Evolving", sections 5.1-5.3 and 5.5 (an indexer without
- * positional encoding scores every historical position; top-K positions are
+ * positional encoding rates all earlier positions; top-K positions are
  * kept; attention over those positions). The page leaves the indexer's form
  * open; it is read here like the block score: for the query at t = seq_lens[b]-1
  *   s(u) = sum_h qi[b][h] . ki[u]        (u < t; fp32: the heads summed left to

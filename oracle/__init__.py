@@ -32,7 +32,7 @@ Citations (page title, section):
                  "Sparse Attention + Linear Backbones: How LLM Long-Context
                  Architectures Are Evolving", sections 5.1-5.3 and 5.5: a
                  lightweight multi-head indexer without positional encoding
-                 scores every historical position, the top-K positions are
+                 rates all earlier positions, the top-K positions are
                  kept, and the main attention runs over those positions only.
                  The page leaves the indexer's form open; the reading here
                  mirrors the block path: s(t, u) = sum over indexer heads h of
