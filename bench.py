@@ -10,8 +10,11 @@ A step is one pass of the whole hot path over one batch of synthetic input:
   decode workloads  : append of one token per sequence, decode selection and
                       split-k decode attention.
 The default workload is the prefill one (batch 1, 32768 tokens, 32/4 heads,
-d 128, block 128, top-k 16); a paged-decode block (batch 32, 131072 cached
-tokens, 32/8 heads, block 64, top-k 32) is measured in the same run.
+d 128, block 128, top-k 16); the other four workloads are measured in the same
+run, one block each in the same JSON line: paged decode ("decode": batch 32,
+131072 cached tokens, 32/8 heads, block 64, top-k 32), 1M-context decode
+("decode_1m": 256 consecutive steps, each appending one token), varlen decode
+("varlen": 64 sequences of 4K-512K tokens) and the tiny fp32 case ("tiny").
 
 Timing: W untimed warm-up steps; the step is then captured in a CUDA graph
 (the library never allocates or synchronises) and K replays are timed between
@@ -66,6 +69,12 @@ def peaks():
 def profile_traffic(kernel: str, src: str):
     """ncu DRAM bytes per launch recorded in profiles/<kernel>*.md, if the kernel
     source still hashes to the recorded value; else None."""
+    return profile_value(kernel, src, "dram_bytes_per_full_launch")
+
+
+def profile_value(kernel: str, src: str, key: str):
+    """A figure `key: value` recorded in profiles/<kernel>*.md, if the kernel
+    source still hashes to the recorded value; else None."""
     pdir = os.path.join(ROOT, "profiles")
     sha = hashlib.sha256(open(os.path.join(ROOT, "block_sparse_gqa_mean_b200", "csrc", src),
                               "rb").read()).hexdigest()[:16]
@@ -76,11 +85,11 @@ def profile_traffic(kernel: str, src: str):
             continue
         vals = {}
         for line in open(os.path.join(pdir, f)):
-            if ":" in line and line.strip().startswith(("source_sha256", "dram_bytes_per_full_launch")):
+            if ":" in line and line.strip().startswith(("source_sha256", key)):
                 k, v = line.strip().split(":", 1)
                 vals[k.strip()] = v.strip().strip("`")
-        if vals.get("source_sha256") == sha and "dram_bytes_per_full_launch" in vals:
-            return float(vals["dram_bytes_per_full_launch"])
+        if vals.get("source_sha256") == sha and key in vals:
+            return float(vals[key])
     return None
 
 
@@ -426,6 +435,185 @@ def run_decode(w, steps, warmup, world, flush_l2):
             "d2h": hout.numel() * 2, "launches_per_step": 1 + 3 + 2}
 
 
+def run_decode_steps(w, world):
+    """Consecutive decode steps (the 1M-context workload): step s sets the
+    length to ctx + s + 1, appends token ctx + s, selects with step s's query
+    and attends. One CUDA graph per step (each holds its own input and output
+    pointers and length), replayed in order; an untimed 256 MB write flushes
+    L2 before every step (the step's ~42 MB would otherwise stay in L2)."""
+    import block_sparse_gqa_mean_b200 as msa
+    dev = torch.device("cuda")
+    cache = fill_decode_cache(w, dev)
+    S, nb = w.steps, w.batch
+    lens = torch.tensor([[w.ctx[b] + s + 1 for b in range(nb)] for s in range(S)],
+                        dtype=torch.int32, device=dev)
+    toks = [workloads.new_tokens(w, s, dev) for s in range(S)]
+    k_all = torch.stack([t[0] for t in toks]).contiguous()         # [S, batch, hkv, d]
+    v_all = torch.stack([t[1] for t in toks]).contiguous()
+    q_all = torch.stack([workloads.queries_decode(w, s, dev) for s in range(S)]).contiguous()
+    out_all = torch.empty_like(q_all)
+    lse_all = torch.empty(S, nb, w.hq, dtype=torch.float32, device=dev)
+    cu = msa.cu_seqlens([1] * nb, dev)
+    idx = torch.empty(nb, w.hkv, w.top_k, dtype=torch.int32, device=dev)
+    ws_sel = torch.empty(max(16, msa.workspace_size(msa.MSA_OP_SELECT, cache, nb, 1, w.top_k)),
+                         dtype=torch.uint8, device=dev)
+    ws_dec = torch.empty(max(16, msa.workspace_size(msa.MSA_OP_DECODE, cache, nb, 1, w.top_k)),
+                         dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def calls(s):
+        def do_len():
+            cache.seq_lens.copy_(lens[s])       # the caller advances the lengths
+        def do_append():
+            msa.build_block_cache(cache, k_all[s], v_all[s], cu, 1)
+        def do_select():
+            msa.select_topk(cache, q_all[s], w.top_k, block_idx=idx, workspace=ws_sel)
+        def do_attn():
+            msa.sparse_attn_decode(cache, q_all[s], idx, out=out_all[s], lse=lse_all[s],
+                                   workspace=ws_dec)
+        return do_len, do_append, do_select, do_attn
+
+    def step_fn(s):
+        fs = calls(s)
+        return lambda: [f() for f in fs]
+
+    graphs = [capture_graph(step_fn(s)) for s in range(S)]   # also runs each step once, in order
+    for g in graphs:                                           # warm-up: the whole run once more
+        g.replay()
+    torch.cuda.synchronize()
+    if cache.device_status() != 0:
+        raise RuntimeError(f"device status {cache.device_status():#x}")
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(S)]
+    barrier(world)
+    torch.cuda.synchronize()
+    with Clocks(torch.cuda.current_device()) as clk:
+        for s in range(S):
+            flush.fill_(s & 0xFF)
+            ev[s][0].record(stream)
+            graphs[s].replay()
+            ev[s][1].record(stream)
+        torch.cuda.synchronize()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    # per-call times on the last step (re-appending its token is idempotent)
+    fl, fa, fs_, ft = calls(S - 1)
+    g_ops = [capture_graph(lambda: (fl(), fa())), capture_graph(fs_), capture_graph(ft)]
+    k_ms = [time_graph(gg, 20, lambda i: flush.fill_(i & 0xFF)) for gg in g_ops]
+
+    # end to end: every step's q and new K/V rows from pinned host memory, its
+    # output back to the host, eager calls
+    hq_, hk, hv = q_all.cpu().pin_memory(), k_all.cpu().pin_memory(), v_all.cpu().pin_memory()
+    hout = torch.empty(out_all.shape, dtype=out_all.dtype).pin_memory()
+    dq, dk, dv = torch.empty_like(q_all[0]), torch.empty_like(k_all[0]), torch.empty_like(v_all[0])
+    dout = torch.empty_like(out_all[0])
+    dlse = torch.empty_like(lse_all[0])
+    e2e = []
+    for s in range(S):
+        flush.fill_(1)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        dq.copy_(hq_[s], non_blocking=True)
+        dk.copy_(hk[s], non_blocking=True)
+        dv.copy_(hv[s], non_blocking=True)
+        cache.seq_lens.copy_(lens[s])
+        msa.build_block_cache(cache, dk, dv, cu, 1)
+        msa.select_topk(cache, dq, w.top_k, block_idx=idx, workspace=ws_sel)
+        msa.sparse_attn_decode(cache, dq, idx, out=dout, lse=dlse, workspace=ws_dec)
+        hout[s].copy_(dout, non_blocking=True)
+        b.record(stream)
+        e2e.append((a, b))
+    torch.cuda.synchronize()
+    e2e_ms = sum(a.elapsed_time(b) for a, b in e2e) / S
+    if not torch.equal(hout.view(torch.int16), out_all.cpu().view(torch.int16)):
+        raise RuntimeError("end-to-end outputs differ from the graph replays")
+    status = cache.device_status()
+    if status != 0:
+        raise RuntimeError(f"device status {status:#x}")
+    return {"step_ms": sum(step_ms) / S, "step_ms_first_last": [step_ms[0], step_ms[-1]],
+            "kernel_ms": k_ms, "clocks": clk.summary(), "e2e_ms": e2e_ms,
+            "h2d": (hq_[0].numel() + hk[0].numel() + hv[0].numel()) * 2,
+            "d2h": hout[0].numel() * 2, "launches_per_step": 1 + 3 + 2, "steps": S}
+
+
+def run_tiny(w, steps, world):
+    """The tiny fp32 workload: prefill of all 1024 rows (append, select,
+    attention; fp32 SIMT kernels), then the decode step that appends token
+    1023 onto 1023 cached tokens and attends."""
+    import block_sparse_gqa_mean_b200 as msa
+    dev = torch.device("cuda")
+    T = w.ctx[0]
+    p = workloads.paging(w)
+    cache = msa.PagedKVCache.allocate(1, p.num_pages, p.max_blocks, w.hq, w.hkv, w.d, w.block,
+                                      w.torch_dtype, dev)
+    cache.page_table.copy_(p.table.to(dev))
+    K = workloads.keys(w, 0, 0, T, dev).contiguous()
+    V = workloads.values(w, 0, 0, T, dev).contiguous()
+    q = workloads.queries_prefill(w, 0, 0, T, dev).contiguous()
+    cu = msa.cu_seqlens([T], dev)
+    cu1 = msa.cu_seqlens([1], dev)
+    idx = torch.empty(T, w.hkv, w.top_k, dtype=torch.int32, device=dev)
+    out = torch.empty_like(q)
+    lse = torch.empty(T, w.hq, dtype=torch.float32, device=dev)
+    didx = torch.empty(1, w.hkv, w.top_k, dtype=torch.int32, device=dev)
+    dout = torch.empty_like(q[:1])
+    dlse = torch.empty(1, w.hq, dtype=torch.float32, device=dev)
+    lens_p = torch.tensor([T], dtype=torch.int32, device=dev)
+    qd = q[T - 1:].contiguous()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def prefill():
+        cache.seq_lens.copy_(lens_p)
+        msa.build_block_cache(cache, K, V, cu, T)
+        msa.select_topk(cache, q, w.top_k, cu_q=cu, max_rows_per_seq=T, block_idx=idx)
+        msa.sparse_attn_prefill(cache, q, idx, cu_q=cu, max_rows_per_seq=T, out=out, lse=lse)
+
+    def decode():
+        cache.seq_lens.copy_(lens_p)                 # token 1023 appended onto 1023 cached
+        msa.build_block_cache(cache, K[T - 1:], V[T - 1:], cu1, 1)
+        msa.select_topk(cache, qd, w.top_k, block_idx=didx)
+        msa.sparse_attn_decode(cache, qd, didx, out=dout, lse=dlse)
+
+    g_p, g_d = capture_graph(prefill), capture_graph(decode)
+    for _ in range(3):
+        g_p.replay()
+        g_d.replay()
+    torch.cuda.synchronize()
+    flush_fn = lambda i: flush.fill_(i & 0xFF)
+    barrier(world)
+    with Clocks(torch.cuda.current_device()) as clk:
+        p_ms = time_graph(g_p, steps, flush_fn)
+        d_ms = time_graph(g_d, steps, flush_fn)
+    if (dout - out[T - 1:]).abs().max().item() > 1e-6:
+        raise RuntimeError("tiny decode differs from prefill row 1023")
+    hq_, hk, hv = q.cpu().pin_memory(), K.cpu().pin_memory(), V.cpu().pin_memory()
+    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(K), torch.empty_like(V)
+    stream = torch.cuda.current_stream()
+    e2e = []
+    for _ in range(steps):
+        flush.fill_(1)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        dq.copy_(hq_, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        cache.seq_lens.copy_(lens_p)
+        msa.build_block_cache(cache, dk, dv, cu, T)
+        msa.select_topk(cache, dq, w.top_k, cu_q=cu, max_rows_per_seq=T, block_idx=idx)
+        msa.sparse_attn_prefill(cache, dq, idx, cu_q=cu, max_rows_per_seq=T, out=out, lse=lse)
+        hout.copy_(out, non_blocking=True)
+        b.record(stream)
+        e2e.append((a, b))
+    torch.cuda.synchronize()
+    if cache.device_status() != 0:
+        raise RuntimeError(f"device status {cache.device_status():#x}")
+    return {"prefill_ms": p_ms, "decode_ms": d_ms, "clocks": clk.summary(),
+            "e2e_ms": sum(a.elapsed_time(b) for a, b in e2e) / steps,
+            "h2d": (hq_.numel() + hk.numel() + hv.numel()) * 4, "d2h": hout.numel() * 4,
+            "launches_per_step": 3}
+
+
 # ---------------------------------------------------------------------------
 # CPU oracle (baseline and reference arm)
 # ---------------------------------------------------------------------------
@@ -443,13 +631,16 @@ def oracle_prefill_sample(w, rows: int):
     return rows, time.perf_counter() - t, oracle.num_threads()
 
 
-def oracle_decode_sample(w, seqs: int):
+def oracle_decode_sample(w, seqs, device="cpu"):
+    """Oracle on the decode step of the listed sequences (the inputs are drawn
+    on `device`, outside the timed region; the oracle runs on the host).
+    Returns (sequences, seconds, threads)."""
     import oracle
     secs, n = 0.0, 0
-    for b in range(seqs):
+    for b in seqs:
         L = w.ctx[b] + 1
-        K = workloads.keys(w, b, 0, L)
-        V = workloads.values(w, b, 0, L)
+        K = workloads.keys(w, b, 0, L, device).cpu()
+        V = workloads.values(w, b, 0, L, device).cpu()
         Q = workloads.queries_decode(w, 0, seqs=[b])
         t = time.perf_counter()
         oracle.forward(Q, K, V, np.array([L - 1]), w.block, w.top_k, w.softmax_scale)
@@ -468,7 +659,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--workload", default="prefill_bf16", choices=list(workloads.ALL))
-    ap.add_argument("--no-decode", action="store_true", help="skip the paged-decode block")
+    ap.add_argument("--no-decode", action="store_true",
+                    help="skip the blocks of the other workloads")
+    ap.add_argument("--blocks", default="decode,decode_1m,varlen,tiny",
+                    help="workload blocks measured after the prefill headline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--oracle-rows", type=int, default=256)
     ap.add_argument("--seq-len", type=int, default=0,
@@ -531,8 +725,7 @@ def main():
             "config": workload_config(w),
         })
         if not args.no_decode and world == 1:
-            wd = workloads.paged_decode_bf16()
-            res["decode"] = decode_block(wd, args, world, pk)
+            res.update(extra_blocks(args, world, pk))
     else:
         res.update(decode_main(w, args, world, pk))
 
@@ -601,8 +794,87 @@ def decode_block(w, args, world, pk):
             "l2": "256 MB write between steps" if flush else "step reads > 126 MB L2, no flush"}
 
 
+def extra_blocks(args, world, pk):
+    """The other four workloads, measured in the same run, one block each."""
+    out = {}
+    for key in [b for b in args.blocks.split(",") if b]:
+        torch.cuda.empty_cache()
+        if key == "decode":
+            w = workloads.paged_decode_bf16()
+            out[key] = decode_block(w, args, world, pk)
+        elif key == "varlen":
+            w = workloads.varlen_decode_bf16()
+            out[key] = decode_block(w, args, world, pk)
+        elif key == "decode_1m":
+            w = workloads.decode_1m_bf16()
+            out[key] = steps_block(w, args, world, pk)
+        elif key == "tiny":
+            w = workloads.tiny_f32()
+            out[key] = tiny_block(w, args, world, pk)
+        else:
+            raise SystemExit(f"unknown block {key}")
+        if not args.no_cpu_baseline and world == 1:
+            out[key]["cpu_baseline"] = cpu_baseline(w, args)
+        out[key]["config"] = workload_config(w)
+    return out
+
+
+def steps_block(w, args, world, pk):
+    """Block of the consecutive-step decode workload (1M context, 256 steps)."""
+    r = run_decode_steps(w, world)
+    ms = max_over_ranks(r["step_ms"], world)
+    nbytes = sum(decode_bytes(w, s) for s in range(w.steps)) / w.steps
+    sel_b, att_b = decode_call_bytes(w, w.steps - 1)
+    sel_ms, att_ms = r["kernel_ms"][1], r["kernel_ms"][2]
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"workload": w.name, "value": w.batch * world / (ms * 1e-3), "unit": "tokens/s",
+            "ms_per_step": ms, "steps": r["steps"], "step_ms_first_last": r["step_ms_first_last"],
+            "hbm_gbs": gbs,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / pk["hbm_gbs"], "traffic": None,
+                         "peak_source": f"{pk['source']} HBM copy",
+                         "scope": "whole decode step (append+select+attention), mean of the "
+                                  f"{w.steps} consecutive steps",
+                         "algorithmic_bytes_per_step": nbytes,
+                         "calls": {
+                             "select_topk": {"bytes": sel_b, "ms": sel_ms,
+                                             "achieved_gbs": sel_b / (sel_ms * 1e-3) / 1e9},
+                             "sparse_attn_decode": {"bytes": att_b, "ms": att_ms,
+                                                    "achieved_gbs": att_b / (att_ms * 1e-3) / 1e9}}},
+            "kernels_ms": {"build_block_cache": r["kernel_ms"][0], "select_topk": sel_ms,
+                           "sparse_attn_decode": att_ms},
+            "e2e": {"value": w.batch * world / (r["e2e_ms"] * 1e-3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
+            "clocks": r["clocks"], "gpu_launches": r["launches_per_step"] * r["steps"],
+            "l2": "256 MB write before every step"}
+
+
+def tiny_block(w, args, world, pk):
+    """Block of the tiny fp32 workload (correctness-sized; fp32 SIMT kernels)."""
+    r = run_tiny(w, args.steps, world)
+    T = w.ctx[0]
+    flops = 4.0 * w.d * attended_pairs(T, w.block, w.top_k) * w.hq
+    ms = max_over_ranks(r["prefill_ms"], world)
+    # fp32 FMA peak from the unit counts: 148 SMs x 128 lanes x 2 flops x clock
+    clk = r["clocks"].get("sm_mhz") or 1965.0
+    peak = 148 * 128 * 2 * clk * 1e6 / 1e12
+    achieved = flops / (ms * 1e-3) / 1e12
+    return {"workload": w.name, "value": T * world / (ms * 1e-3), "unit": "tokens/s",
+            "ms_per_step": ms, "decode_ms": r["decode_ms"],
+            "roofline": {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "traffic": None,
+                         "peak_source": "fp32 FMA lanes x clock (148 x 128 x 2 x sampled SM MHz)",
+                         "scope": "whole prefill step (append+select+attention; 1024 rows, "
+                                  "latency-bound at this size)",
+                         "algorithmic_flops_per_step": flops},
+            "e2e": {"value": T * world / (r["e2e_ms"] * 1e-3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
+            "clocks": r["clocks"], "gpu_launches": r["launches_per_step"] * args.steps,
+            "l2": "256 MB write between steps"}
+
+
 def decode_main(w, args, world, pk):
-    d = decode_block(w, args, world, pk)
+    d = steps_block(w, args, world, pk) if w.steps > 1 else decode_block(w, args, world, pk)
     return {"metric": METRIC, "value": d["value"], "unit": "tokens/s", "ms_per_step": d["ms_per_step"],
             "roofline": d["roofline"], "kernels_ms": d["kernels_ms"], "e2e": d["e2e"],
             "clocks": d["clocks"], "gpu_launches": d["gpu_launches"],
@@ -619,7 +891,9 @@ def workload_config(w):
     c = {"workload": w.name, "batch": w.batch, "q_heads": w.hq, "kv_heads": w.hkv,
          "head_dim": w.d, "block": w.block, "top_k": w.top_k}
     if w.kind == "prefill":
-        c.update({"seq_len": w.ctx[0], "l2": "inputs 0.7 GB per step > 126 MB L2, no flush"})
+        c.update({"seq_len": w.ctx[0],
+                  "l2": ("256 MB write between steps" if w.name == "tiny_f32"
+                         else "inputs 0.7 GB per step > 126 MB L2, no flush")})
     else:
         c.update({"context_mean": float(np.mean(w.ctx)),
                   "l2": ("256 MB write between steps" if decode_flush(w)
@@ -633,11 +907,22 @@ def cpu_baseline(w, args):
         return {"value": n / secs, "unit": "tokens/s", "cores": thr, "kind": "oracle",
                 "sample": f"{n} query rows spread over the {w.ctx[0]}-token sequence, plus the "
                           f"block cache of the whole sequence, fp64, OpenMP"}
-    seqs = min(w.batch, 2)
-    n, secs, thr = oracle_decode_sample(w, seqs)
+    seqs = sample_seqs(w)
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    n, secs, thr = oracle_decode_sample(w, seqs, dev)
     return {"value": n / secs, "unit": "tokens/s", "cores": thr, "kind": "oracle",
-            "sample": f"{n} of {w.batch} sequences' decode step (block cache of the whole "
-                      f"context + selection + attention), fp64, OpenMP"}
+            "sample": f"{n} of {w.batch} sequences' decode step (lengths "
+                      f"{[w.ctx[b] + 1 for b in seqs]}: block cache of the whole context + "
+                      f"selection + attention), fp64, OpenMP"}
+
+
+def sample_seqs(w):
+    """Sequences of the bounded CPU sample of a decode workload: the first two,
+    or for varied lengths the one closest to the mean length."""
+    if len(set(w.ctx)) > 1:
+        mean = float(np.mean(w.ctx))
+        return [int(np.argmin([abs(L - mean) for L in w.ctx]))]
+    return list(range(min(w.batch, 2 if w.ctx[0] <= (1 << 17) else 1)))
 
 
 def reference_arm(w, args):
@@ -647,7 +932,7 @@ def reference_arm(w, args):
         if w.kind == "prefill":
             n, secs, thr = oracle_prefill_sample(w, max(8, args.oracle_rows // 4))
         else:
-            n, secs, thr = oracle_decode_sample(w, 1)
+            n, secs, thr = oracle_decode_sample(w, sample_seqs(w)[:1])
         if i >= args.warmup:
             steps.append((n, secs))
     n = sum(s[0] for s in steps)

@@ -47,6 +47,11 @@ inline cudaError_t launch_pdl(void (*kernel)(P...), dim3 grid, dim3 block, size_
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<A>(args)...);
 }
 
+// Host-side checks shared by the decode attention entry points (msa_api.cu).
+msa_status_t check_decode_args(const msa_paged_kv_t* kv, const void* q, const int32_t* block_idx,
+                               int32_t top_k, float softmax_scale, const void* out,
+                               const float* lse);
+
 __device__ __forceinline__ void report(uint32_t* status, uint32_t bits) {
   if (status) atomicOr(status, bits);
 }

@@ -56,7 +56,10 @@ extern "C" msa_status_t msa_sparse_attn_decode_noalloc(const msa_paged_kv_t* kv,
                                                        const int32_t* block_idx, int32_t top_k,
                                                        float softmax_scale, void* out, float* lse,
                                                        msa_stream_t stream) {
-  if (!kv) return MSA_ERR_INVALID_ARG;
+  // bad arguments are reported as such, before the scratch array is looked up
+  const msa_status_t s =
+      msa::check_decode_args(kv, q, block_idx, top_k, softmax_scale, out, lse);
+  if (s != MSA_OK) return s;
   const size_t need = msa_workspace_size(MSA_OP_DECODE, kv, kv->batch, 1, top_k);
   if (need > kNoAllocScratchBytes) return MSA_ERR_WORKSPACE;
   void* scratch = scratch_on_current_device();

@@ -104,6 +104,20 @@ static bool use_decode_splitk(const msa_paged_kv_t* kv) {
 
 static msa_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? MSA_OK : MSA_ERR_CUDA; }
 
+// Host-side checks of the decode attention arguments other than the
+// workspace; every decode attention entry point runs them before anything else.
+msa_status_t check_decode_args(const msa_paged_kv_t* kv, const void* q, const int32_t* block_idx,
+                               int32_t top_k, float softmax_scale, const void* out,
+                               const float* lse) {
+  msa_status_t s = check_kv(kv);
+  if (s != MSA_OK) return s;
+  if (top_k < 1 || top_k > 256) return MSA_ERR_UNSUPPORTED;
+  if (!q || !block_idx || !out || !aligned(q, 16) || !aligned(out, 16) || !aligned(block_idx, 4) ||
+      (lse && !aligned(lse, 4)) || !(softmax_scale > 0.f))
+    return MSA_ERR_INVALID_ARG;
+  return MSA_OK;
+}
+
 }  // namespace msa
 
 using namespace msa;
@@ -211,12 +225,8 @@ static msa_status_t attn_decode(const msa_paged_kv_t* kv, const void* q, const i
                                 int32_t top_k, float softmax_scale, gate_t gate, void* out,
                                 float* lse, void* workspace, size_t workspace_bytes,
                                 msa_stream_t stream) {
-  msa_status_t s = check_kv(kv);
+  msa_status_t s = check_decode_args(kv, q, block_idx, top_k, softmax_scale, out, lse);
   if (s != MSA_OK) return s;
-  if (top_k < 1 || top_k > 256) return MSA_ERR_UNSUPPORTED;
-  if (!q || !block_idx || !out || !aligned(q, 16) || !aligned(out, 16) || !aligned(block_idx, 4) ||
-      (lse && !aligned(lse, 4)) || !(softmax_scale > 0.f))
-    return MSA_ERR_INVALID_ARG;
   cudaStream_t st = (cudaStream_t)stream;
   if (use_decode_splitk(kv)) {
     const int sms = num_sms();

@@ -21,9 +21,13 @@
  * Conventions for every entry point
  * ---------------------------------
  *  - All tensor arguments are DEVICE pointers owned by the caller; the library
- *    never allocates, frees or synchronises, and keeps no mutable global state
- *    (entry points may be called from several host threads on different
- *    streams). Every call is asynchronous on `stream`.
+ *    never allocates, frees or synchronises. Except for
+ *    msa_sparse_attn_decode_noalloc, it keeps no mutable global state, so
+ *    those entry points may be called from several host threads on different
+ *    streams. msa_sparse_attn_decode_noalloc is the one exception: it keeps
+ *    its scratch in one library-owned device array per GPU, and its calls
+ *    must not overlap on the GPU (see its own comment). Every call is
+ *    asynchronous on `stream`.
  *  - Host-side validation runs before any launch. It returns
  *    MSA_ERR_INVALID_ARG for null or misaligned pointers (16-byte alignment is
  *    required for every tensor) and inconsistent sizes, MSA_ERR_UNSUPPORTED
@@ -265,6 +269,8 @@ msa_status_t msa_sparse_attn_decode_gated(const msa_paged_kv_t* kv, const void* 
  * Same arguments and results as msa_sparse_attn_decode minus the workspace:
  * the split-k partials go to one 8 MiB device array inside libmsa.so, which
  * every GPU that loads the library keeps until the process exits.
+ *  - Bad arguments give the same status as msa_sparse_attn_decode, checked
+ *    before anything else (the array is not looked up).
  *  - Returns MSA_ERR_WORKSPACE, launching nothing, when the problem needs more
  *    than 8 MiB, i.e. when msa_workspace_size(MSA_OP_DECODE, kv, batch, 1,
  *    top_k) > 8 MiB (about batch * num_q_heads * splits * 516 bytes).

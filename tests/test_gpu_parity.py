@@ -184,6 +184,12 @@ def test_chunked_prefill_matches_full():
     torch.cuda.synchronize()
     assert torch.equal(idx, full[2][T0:])
     compare(out, full[4][T0:].float().cpu().double().numpy(), "bf16")
+    # and the chunk's selection against the oracle at positions T0 .. T-1
+    pos = np.arange(T0, T)
+    orc = oracle_rows(w, 0, T, pos, q.cpu())
+    check_selection(idx.cpu().numpy(), orc, pos, w.top_k, w.block)
+    same = (idx.cpu().numpy() == orc["idx"]).all(-1).all(-1)
+    compare(out[torch.from_numpy(same).to(DEV)], orc["out"][same], "bf16")
 
 
 def test_prefill_batch_varlen_chunked_and_index_edges():
@@ -223,6 +229,11 @@ def test_prefill_batch_varlen_chunked_and_index_edges():
         pos = np.arange(first[b], w.ctx[b])
         sl = slice(r0, r0 + n[b])
         qb = q[sl].cpu()
+        # selection of every row (the chunk's rows sit after cached tokens)
+        # against the oracle's own top-k at those positions
+        sel = check_selection(gi[sl], oracle_rows(w, b, w.ctx[b], pos, qb), pos, w.top_k,
+                              w.block)
+        assert sel["protected_frac"] > 0.3
         orc = oracle_rows(w, b, w.ctx[b], pos, qb, idx=gi[sl])
         compare(out[sl], orc["out"], w.dtype)
         assert np.abs(lse[sl].cpu().double().numpy() - orc["lse"]).max() < 2e-3

@@ -34,7 +34,12 @@ def _index_pages(w, p, lens):
     return ki
 
 
-@pytest.mark.parametrize("top_k", [1, 256, 6000])
+# sequences (of 3) whose oracle gap is >= GAP_MIN, so that their kept list must
+# be bit-exact; read off the seeded inputs with the oracle alone (CPU)
+MIN_PROTECTED = {1: 3, 16: 3, 64: 3, 256: 2, 2048: 3, 6000: 3}
+
+
+@pytest.mark.parametrize("top_k", sorted(MIN_PROTECTED))
 def test_token_decode_selection_and_attention(top_k):
     w = workloads.paged_decode_bf16(batch=3, ctx=(3000, 5000, 4096))
     p = workloads.paging(w)
@@ -51,6 +56,7 @@ def test_token_decode_selection_and_attention(top_k):
     gi = idx.cpu().numpy()
     oidx_all, refs = [], []
     found = [0, 0]
+    protected = 0
     for b in range(w.batch):
         L = after[b]
         pos = np.array([L - 1])
@@ -62,6 +68,7 @@ def test_token_decode_selection_and_attention(top_k):
         assert kept == sorted(set(kept)) and kept[-1] == L - 1
         assert len(kept) == min(top_k, L) and np.all(row[len(kept):] == -1)
         if gap[0] >= GAP_MIN:
+            protected += 1
             assert np.array_equal(row, oidx[0])
         elif not np.array_equal(row, oidx[0]):
             earlier = [u for u in kept if u != L - 1]
@@ -74,8 +81,9 @@ def test_token_decode_selection_and_attention(top_k):
         O, _ = oracle.attend_tokens(q[b:b + 1].cpu(), K, V, pos, oidx, w.softmax_scale)
         oidx_all.append(oidx)
         refs.append(O)
-    if top_k == 256:
-        assert found[0] >= 0.75 * found[1], found
+    assert protected >= MIN_PROTECTED[top_k], protected
+    if top_k >= 256:
+        assert found[0] == found[1], found   # every planted position is kept
     oi = torch.from_numpy(np.concatenate(oidx_all)).to(DEV)
     out, lse = msa.sparse_attn_decode_tokens(cache, q, oi)
     torch.cuda.synchronize()

@@ -3,56 +3,148 @@
 msa_sparse_attn_decode_noalloc serves callers that cannot allocate device
 memory at the call (a plugin inside a framework that owns the memory pool, an
 allocator-free latency loop): it keeps its split-k scratch in a fixed 8 MiB
-device array inside the library. This file is collected last on purpose, so a
-run that stops at the first failure has run every other test first; it also
-passes on its own in a fresh process (the first call sets up the array's
-device address).
+device array inside the library. It runs the same kernels as
+msa_sparse_attn_decode, so its outputs must equal the regular entry point's
+bit for bit, call after call, and a call must not change the device's free
+memory. This file is collected last on purpose, so a run that stops at the
+first failure has run every other test first; it also passes on its own in a
+fresh process (the first call sets up the array's device address).
 """
 import ctypes
 
+import numpy as np
 import pytest
 import torch
 
 import block_sparse_gqa_mean_b200 as msa
 import workloads
-from msa_harness import TOL, append, fill_context, new_cache
+from msa_harness import append, fill_context, new_cache
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
+SCRATCH_BYTES = 8 << 20
 
 
-def _decode_case():
-    w = workloads.paged_decode_bf16(batch=4, ctx=(3000, 4095, 4096, 5000))
+def _decode_case(batch=4, ctx=(3000, 4095, 4096, 5000)):
+    w = workloads.paged_decode_bf16(batch=batch, ctx=ctx)
     p = workloads.paging(w)
     cache = new_cache(w, p)
-    lens = fill_context(cache, w)
+    lens = fill_context(cache, w) if batch <= 8 else _fill_all(cache, w)
     append(cache, w, lens, [L + 1 for L in lens])
     q = workloads.queries_decode(w, 0, DEV)
     idx, _ = msa.select_topk(cache, q, w.top_k)
     return w, cache, q, idx
 
 
-def test_noalloc_decode_matches_regular_entry_point_twice():
-    w, cache, q, idx = _decode_case()
+def _fill_all(cache, w):
+    append(cache, w, [0] * w.batch, list(w.ctx))
+    return list(w.ctx)
+
+
+def _noalloc(cache, q, idx, top_k, out, lse):
+    lib = msa.load_library()
+    kv = cache.struct()
+    return lib.msa_sparse_attn_decode_noalloc(ctypes.byref(kv), q.data_ptr(), idx.data_ptr(),
+                                              top_k, 1.0 / 128 ** 0.5, out.data_ptr(),
+                                              lse.data_ptr(), None)
+
+
+def _same_bits(a, b):
+    return torch.equal(a.view(torch.int16) if a.dtype == torch.bfloat16 else a.view(torch.int32),
+                       b.view(torch.int16) if b.dtype == torch.bfloat16 else b.view(torch.int32))
+
+
+def _check_twice_against_regular(w, cache, q, idx):
     ref, ref_lse = msa.sparse_attn_decode(cache, q, idx)
     torch.cuda.synchronize()
     for _ in range(2):  # two calls in a row share the library's scratch array
         out = torch.full_like(q, float("nan"))
         lse = torch.full((q.shape[0], q.shape[1]), float("nan"), device=DEV)
-        msa.sparse_attn_decode_noalloc(cache, q, idx, out, lse)
+        assert _noalloc(cache, q, idx, w.top_k, out, lse) == msa.MSA_OK
         torch.cuda.synchronize()
-        err = (out.float() - ref.float()).abs().max().item()
-        rel = ((out.float() - ref.float()).norm() / ref.float().norm()).item()
-        assert err <= TOL["bf16"]["max_abs"] and rel <= TOL["bf16"]["rel_l2"], (err, rel)
-        assert (lse - ref_lse).abs().max().item() <= 1e-4
+        assert _same_bits(out, ref) and _same_bits(lse, ref_lse)
     assert cache.device_status() == 0
 
 
-def test_noalloc_rejects_problems_beyond_its_scratch():
+def test_noalloc_decode_matches_regular_entry_point_twice():
     w, cache, q, idx = _decode_case()
+    _check_twice_against_regular(w, cache, q, idx)
+
+
+def test_noalloc_allocates_nothing():
+    w, cache, q, idx = _decode_case()
+    out = torch.empty_like(q)
+    lse = torch.empty(q.shape[0], q.shape[1], device=DEV)
+    assert _noalloc(cache, q, idx, w.top_k, out, lse) == msa.MSA_OK  # address set-up done
+    torch.cuda.synchronize()
+    alloc0 = torch.cuda.memory_allocated()
+    free0, _ = torch.cuda.mem_get_info()
+    for _ in range(3):
+        assert _noalloc(cache, q, idx, w.top_k, out, lse) == msa.MSA_OK
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert torch.cuda.memory_allocated() == alloc0
+    assert free1 == free0
+
+
+def _largest_batch_within_scratch(cache, top_k):
+    """The largest batch whose split-k partials fit the 8 MiB array, found with
+    the library's own workspace arithmetic on a copy of the descriptor."""
+    lib = msa.load_library()
     kv = cache.struct()
-    kv.batch = 100000  # split-k partials would need far more than 8 MiB
+
+    def need(batch):
+        kv.batch = batch
+        return int(lib.msa_workspace_size(msa.MSA_OP_DECODE, ctypes.byref(kv), batch, 1, top_k))
+
+    lo, hi = 1, 1
+    while need(hi) <= SCRATCH_BYTES:
+        lo, hi = hi, hi * 2
+    while hi - lo > 1:
+        mid = (lo + hi) // 2
+        lo, hi = (mid, hi) if need(mid) <= SCRATCH_BYTES else (lo, mid)
+    return lo, need(lo), need(lo + 1)
+
+
+def test_noalloc_at_the_scratch_limit():
+    probe = new_cache(workloads.paged_decode_bf16(batch=1, ctx=(64,)),
+                      workloads.paging(workloads.paged_decode_bf16(batch=1, ctx=(64,))))
+    top_k = workloads.paged_decode_bf16().top_k
+    batch, under, over = _largest_batch_within_scratch(probe, top_k)
+    assert under <= SCRATCH_BYTES < over
+    assert under > SCRATCH_BYTES - (64 << 10)    # just under the limit
+    rng = np.random.default_rng(3)
+    ctx = tuple(int(x) for x in rng.integers(100, 700, batch))
+    w, cache, q, idx = _decode_case(batch=batch, ctx=ctx)
+    assert msa.workspace_size(msa.MSA_OP_DECODE, cache, batch, 1, w.top_k) == under
+    _check_twice_against_regular(w, cache, q, idx)
+    # one sequence more does not fit: refused before anything is launched
+    kv = cache.struct()
+    kv.batch = batch + 1
+    out = torch.empty_like(q)
     lib = msa.load_library()
     st = lib.msa_sparse_attn_decode_noalloc(ctypes.byref(kv), q.data_ptr(), idx.data_ptr(),
-                                            w.top_k, 0.0884, q.data_ptr(), None, None)
+                                            w.top_k, 0.0884, out.data_ptr(), None, None)
     assert st == msa.MSA_ERR_WORKSPACE
+
+
+def test_noalloc_rejects_bad_arguments_first():
+    w, cache, q, idx = _decode_case()
+    lib = msa.load_library()
+    kv = cache.struct()
+    out = torch.empty_like(q)
+    # a null query or a zero scale is an argument error, not a scratch problem
+    assert lib.msa_sparse_attn_decode_noalloc(ctypes.byref(kv), None, idx.data_ptr(), w.top_k,
+                                              0.0884, out.data_ptr(), None, None) == \
+        msa.MSA_ERR_INVALID_ARG
+    assert lib.msa_sparse_attn_decode_noalloc(ctypes.byref(kv), q.data_ptr(), idx.data_ptr(),
+                                              w.top_k, 0.0, out.data_ptr(), None, None) == \
+        msa.MSA_ERR_INVALID_ARG
+    assert lib.msa_sparse_attn_decode_noalloc(ctypes.byref(kv), q.data_ptr(), idx.data_ptr(),
+                                              0, 0.0884, out.data_ptr(), None, None) == \
+        msa.MSA_ERR_UNSUPPORTED
+    big = cache.struct()
+    big.batch = 100000  # split-k partials would need far more than 8 MiB
+    assert lib.msa_sparse_attn_decode_noalloc(ctypes.byref(big), q.data_ptr(), idx.data_ptr(),
+                                              w.top_k, 0.0884, q.data_ptr(), None, None) == \
+        msa.MSA_ERR_WORKSPACE
