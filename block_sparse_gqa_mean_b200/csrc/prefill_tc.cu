@@ -572,12 +572,14 @@ __global__ void __launch_bounds__(192, 1) prefill_tc_kernel(
           for (int xx = 0; xx < 32; ++xx) s[c * 32 + xx] = __uint_as_float(v[xx]);
         }
         tc_wait_ld();
+        tc_tie(s);
       } else if (mode == 1) {
         uint32_t v[B / 2];
         tc_ld16x2(lane_base + ((uint32_t)(hv * 16) << 16) + COL_S, v);
+        tc_wait_ld();
+        tc_tie(v);
 #pragma unroll
         for (int xx = 0; xx < B / 2; ++xx) s[xx] = __uint_as_float(v[xx]);
-        tc_wait_ld();
       }
       tc_fence_before();
       mbar_arrive(&s_free);                        // S is in registers: the next S may start
@@ -635,6 +637,7 @@ __global__ void __launch_bounds__(192, 1) prefill_tc_kernel(
           uint32_t v[32];
           tc_ld32(lane_base + COL_O + c * 32, v);
           tc_wait_ld();
+          tc_tie(v);
 #pragma unroll
           for (int xx = 0; xx < 32; ++xx) v[xx] = __float_as_uint(__uint_as_float(v[xx]) * alpha);
           tc_st32(lane_base + COL_O + c * 32, v);
@@ -668,9 +671,10 @@ __global__ void __launch_bounds__(192, 1) prefill_tc_kernel(
         uint32_t pv[B / 4];
         exp_pack<B / 4>(s, sl2, neg_m, pv, lsum2);
         tc_st16x2(lane_base + ((uint32_t)(hv * 16) << 16) + COL_P + pb * 64, pv);
+        uint32_t zero[B / 4];
 #pragma unroll
-        for (int xx = 0; xx < B / 4; ++xx) pv[xx] = 0u;
-        tc_st16x2(lane_base + ((uint32_t)((1 - hv) * 16) << 16) + COL_P + pb * 64, pv);
+        for (int xx = 0; xx < B / 4; ++xx) zero[xx] = 0u;
+        tc_st16x2(lane_base + ((uint32_t)((1 - hv) * 16) << 16) + COL_P + pb * 64, zero);
         const float lh = __uint_as_float((uint32_t)lsum2) + __uint_as_float((uint32_t)(lsum2 >> 32));
         const float lp = __shfl_xor_sync(0xffffffffu, lh, 16);
         if (owner && sel) l_run += lh + lp;
@@ -699,6 +703,7 @@ __global__ void __launch_bounds__(192, 1) prefill_tc_kernel(
         uint32_t v[32];
         tc_ld32(lane_base + COL_O + c * 32, v);
         tc_wait_ld();
+        tc_tie(v);
         if (row_ok && gate.g) {  // fused output gate: O = g A + (1 - g) X, one rounding
 #pragma unroll
           for (int xx = 0; xx < 32; ++xx)

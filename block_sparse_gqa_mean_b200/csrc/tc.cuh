@@ -34,6 +34,26 @@ __device__ __forceinline__ void tc_commit(uint64_t* bar) {
 }
 
 __device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// The destination registers of tcgen05.ld hold their values only once
+// tcgen05.wait::ld has returned, but nothing in the inline assembly tells the
+// compiler so: it could move a use of those registers above the wait. After
+// the wait, tc_tie passes the registers through an empty volatile asm (which
+// keeps its place after the wait), so every use depends on it.
+template <int N>
+__device__ __forceinline__ void tc_tie(uint32_t (&r)[N]) {
+#pragma unroll
+  for (int i = 0; i < N; i += 8)
+    asm volatile("" : "+r"(r[i]), "+r"(r[i + 1]), "+r"(r[i + 2]), "+r"(r[i + 3]), "+r"(r[i + 4]),
+                 "+r"(r[i + 5]), "+r"(r[i + 6]), "+r"(r[i + 7]));
+}
+template <int N>
+__device__ __forceinline__ void tc_tie(float (&r)[N]) {
+#pragma unroll
+  for (int i = 0; i < N; i += 8)
+    asm volatile("" : "+f"(r[i]), "+f"(r[i + 1]), "+f"(r[i + 2]), "+f"(r[i + 3]), "+f"(r[i + 4]),
+                 "+f"(r[i + 5]), "+f"(r[i + 6]), "+f"(r[i + 7]));
+}
 __device__ __forceinline__ void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // 32 lanes x 32 consecutive 32-bit columns: thread i of the warp gets lane i.

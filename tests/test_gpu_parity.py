@@ -88,6 +88,10 @@ PREFILL_CASES = [
     ("g16_b128", dict(ctx=(900,), hq=64, hkv=4, top_k=3)),
     ("g8_b64", dict(ctx=(700,), block=64, top_k=5)),
     ("g4_simt", dict(ctx=(500,), hq=16, hkv=4, top_k=3)),
+    # no planted blocks: selections differ from token to token, so tiles walk
+    # wide unions and the softmax takes its one-half-of-a-warp path often
+    ("g16_b128_unplanted", dict(ctx=(2048,), hq=64, hkv=4, top_k=6, planted=(0, 0))),
+    ("g8_b128_unplanted", dict(ctx=(4096,), top_k=8, planted=(0, 0))),
 ]
 
 
