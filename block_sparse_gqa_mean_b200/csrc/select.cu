@@ -51,10 +51,10 @@ __host__ __device__ inline int pass1_sc(int hkv) {
   while (sc > 1 && sc * hkv > kPass1Threads) sc >>= 1;
   return sc;
 }
-// one stage: SC padded page copies, then the item's qbar rows; 128-byte multiple
-__host__ __device__ inline int pass1_stage_bytes(int hkv, int D) {
-  const int page = hkv * D * 4;
-  return (pass1_sc(hkv) * (page + 16) + page + 127) & ~127;
+// one stage: SC padded page copies (the item's groups of each candidate); 128-byte multiple
+__host__ __device__ inline int pass1_stage_bytes(int hg, int D) {
+  const int page = hg * D * 4;
+  return (pass1_sc(hg) * (page + 16) + 127) & ~127;
 }
 
 // qbar[i..i+VEC) = q_{gG}[i] + q_{gG+1}[i] + ... (left to right over the heads)
@@ -295,30 +295,6 @@ __global__ void __launch_bounds__(256, KMAX <= 16 ? 3 : 1) select_rows_kernel(
 // ---------------------------------------------------------------------------
 // select_decode
 // ---------------------------------------------------------------------------
-// qbar of every (sequence, group) for decode: the group's query heads summed
-// left to right in fp32, the same order load_qbar_vec uses. [batch][hkv][D].
-// One CTA per (group, sequence), one thread per coordinate, all head loads in
-// flight together.
-template <typename T, int D>
-__global__ void __launch_bounds__(D) select_decode_qbar(const T* __restrict__ q, int hq, int hkv,
-                                                       float* __restrict__ qbar,
-                                                       unsigned int* __restrict__ next_item) {
-  pdl_wait();
-  const int g = blockIdx.x, b = blockIdx.y, i = threadIdx.x;
-  if (g == 0 && b == 0 && i == 0) *next_item = 0u;  // pass 1's work counter
-  const int G = hq / hkv;
-  const T* p = q + ((size_t)b * hq + (size_t)g * G) * D + i;
-  float v[16];
-#pragma unroll
-  for (int h = 0; h < 16; ++h) v[h] = h < G ? to_f32(p[(size_t)h * D]) : 0.f;
-  float a = v[0];
-#pragma unroll
-  for (int h = 1; h < 16; ++h)
-    if (h < G) a = __fadd_rn(a, v[h]);
-  qbar[((size_t)b * hkv + g) * D + i] = a;
-  pdl_release();
-}
-
 __device__ __forceinline__ uint64_t shfl_xor_u64(uint64_t v, int m) {
   const uint32_t lo = __shfl_xor_sync(0xffffffffu, (uint32_t)v, m);
   const uint32_t hi = __shfl_xor_sync(0xffffffffu, (uint32_t)(v >> 32), m);
@@ -327,27 +303,31 @@ __device__ __forceinline__ uint64_t shfl_xor_u64(uint64_t v, int m) {
 
 // Pass 1 of decode selection. An item is (sequence b, chunk c of 64 candidate
 // blocks, subset gs of hg consecutive KV groups); items are numbered over the
-// non-empty chunks and claimed by persistent CTAs from a counter that the
-// qbar kernel zeroes, so faster CTAs take more items. The block cache
-// keeps all groups of a page together, so one bulk copy brings one candidate
-// for the item's hg groups (hg * D fp32, 2 KB for 4 groups of d 128). An item
-// is streamed in KPL steps of SC = 64 / KPL candidates through an NST-stage
-// ring of shared memory.
-//   * warp 4 (producer) reads the page-table entries one step ahead, and per
-//     step issues the page copies plus a copy of the item's qbar rows, all
-//     completing on the stage's `full` mbarrier;
-//   * warps 0-3 (consumers): thread t scores candidate t % SC of the step for
-//     group gs * hg + t / SC with the canonical fp32 fma chain, keeps the key in
-//     register slot `step`, and the warp releases the stage on `empty`. After
-//     the item's last step the SC lanes of a group hold its 64 keys (KPL
-//     each) and sort them with a bitonic network (in-register strides below
-//     KPL, shuffles above); element e of the sorted order is rank e.
-template <int D, int KPL, int NST>
+// non-empty chunks and taken round-robin by the persistent CTAs (CTA i takes
+// items i, i + grid, ...; the items are equal in size but for each sequence's
+// last chunk). The block cache keeps all groups of a page together, so one
+// bulk copy brings one candidate for the item's hg groups (hg * D fp32, 2 KB
+// for 4 groups of d 128). An item is streamed in KPL steps of SC = 64 / KPL
+// candidates through an NST-stage ring of shared memory.
+//   * warp 4 (producer) reads the page-table entries one step ahead and per
+//     step issues the page copies, completing on the stage's `full` mbarrier;
+//     with an item's first step it also copies the item's raw query rows (its
+//     hg groups' G heads each) into `qraw`, completing on `qfull`;
+//   * warps 0-3 (consumers): at the start of an item they sum each group's
+//     query heads into qbar (fp32, left to right over the heads: the same order
+//     as every other selection path), then thread t scores candidate t % SC of
+//     each step for group gs * hg + t / SC with the canonical fp32 fma chain,
+//     keeps the key in register slot `step`, and the warp releases the stage
+//     on `empty`. After the item's last step the SC lanes of a group hold its
+//     64 keys (KPL each) and sort them with a bitonic network (in-register
+//     strides below KPL, shuffles above); element e of the sorted order is
+//     rank e.
+template <typename T, int D, int KPL, int NST>
 __global__ void __launch_bounds__(kPass1Threads + 32, 1) select_decode_pass1(
-    const float* __restrict__ qbar_all, const float* __restrict__ centroids,
+    const T* __restrict__ q, const float* __restrict__ centroids,
     const int32_t* __restrict__ page_table, const int32_t* __restrict__ seq_lens, uint32_t* status,
-    int batch, int hkv, int hg, int B, int num_pages, int max_blocks, int kw, int nchunks,
-    uint64_t* __restrict__ ws, unsigned int* __restrict__ next_item) {
+    int batch, int hq, int hkv, int hg, int B, int num_pages, int max_blocks, int kw, int nchunks,
+    uint64_t* __restrict__ ws) {
   constexpr int SC = kDecChunk / KPL;         // candidates per step = lanes per group
   constexpr int NCW = kPass1Threads / 32;     // consumer warps
   constexpr int NW = NCW + 1;
@@ -356,15 +336,20 @@ __global__ void __launch_bounds__(kPass1Threads + 32, 1) select_decode_pass1(
   extern __shared__ __align__(128) unsigned char smem_raw[];
   __shared__ __align__(8) uint64_t full[NST];
   __shared__ __align__(8) uint64_t empty[NST];
+  __shared__ __align__(8) uint64_t qfull, qempty, qready;
   __shared__ int s_item[NST][3];  // (b, c, gs) of the step held by each stage
   __shared__ uint32_t s_valid[NST];  // bit k: candidate k of the step was copied
   __shared__ int wsum[NW];
+  const int G = hq / hkv;
   const int hsplit = hkv / hg;                 // items per (sequence, chunk)
   const uint32_t page_bytes = (uint32_t)hg * D * 4;  // the item's groups of one page
+  const uint32_t q_bytes = (uint32_t)hg * G * D * sizeof(T);  // the item's raw query rows
   const int pstride = (int)page_bytes + 16;   // padded: conflict-free float4 reads
   const int stage_bytes = pass1_stage_bytes(hg, D);
-  int* pre = reinterpret_cast<int*>(smem_raw + (size_t)NST * stage_bytes);  // [batch + 1]
-  int* ncs = pre + batch + 1;                                                // [batch]
+  T* qraw = reinterpret_cast<T*>(smem_raw + (size_t)NST * stage_bytes);
+  float* qbar2 = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(qraw) + q_bytes);  // [2][hg][D]
+  int* pre = reinterpret_cast<int*>(qbar2 + 2 * hg * D);                                       // [batch + 1]
+  int* ncs = pre + batch + 1;                                                                  // [batch]
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
   if (tid == 0) {
@@ -372,6 +357,9 @@ __global__ void __launch_bounds__(kPass1Threads + 32, 1) select_decode_pass1(
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], NCW);
     }
+    mbar_init(&qfull, 1);
+    mbar_init(&qempty, NCW);
+    mbar_init(&qready, kPass1Threads);
     mbar_fence_init();
   }
   pdl_wait();
@@ -415,13 +403,6 @@ __global__ void __launch_bounds__(kPass1Threads + 32, 1) select_decode_pass1(
 
   if (warp == NCW) {
     // ------------------------------ producer ------------------------------
-    // items are claimed from a shared counter when their first step is fetched
-    auto claim = [&]() {
-      unsigned int v = 0;
-      if (lane == 0) v = atomicAdd(next_item, 1u);
-      v = __shfl_sync(0xffffffffu, v, 0);
-      return v < (unsigned int)total_items ? (int)v : -1;
-    };
     int cur_b = 0, cur_c = 0, cur_gs = 0;
     // locate item `it` (sets cur_*); returns this lane's page entry for step `sub`
     auto fetch = [&](int it, int sub) {
@@ -437,9 +418,9 @@ __global__ void __launch_bounds__(kPass1Threads + 32, 1) select_decode_pass1(
       const int j = cur_c * kDecChunk + sub * SC + lane;
       return (lane < SC && j < ncs[lo]) ? page_table[(size_t)lo * max_blocks + j] : kNoCand;
     };
-    int it = claim(), sub = 0;
+    int it = (int)blockIdx.x < total_items ? (int)blockIdx.x : -1, sub = 0;
     int pg = it >= 0 ? fetch(it, 0) : kNoCand;
-    int n = 0;
+    int n = 0, items = 0;
     for (;; ++n) {
       const int s = n % NST;
       if (n >= NST &&
@@ -455,6 +436,20 @@ __global__ void __launch_bounds__(kPass1Threads + 32, 1) select_decode_pass1(
         ++n;
         break;
       }
+      if (sub == 0) {
+        // the item's query rows, once the consumers are done with the last item's
+        if (items > 0 &&
+            !__all_sync(0xffffffffu, mbar_wait(&qempty, (uint32_t)(items - 1) & 1u))) {
+          if (lane == 0) report(status, MSA_DEV_TIMEOUT);
+          break;
+        }
+        if (lane == 0) {
+          mbar_expect_tx(&qfull, q_bytes);
+          bulk_load_1d(qraw, q + ((size_t)cur_b * hq + (size_t)cur_gs * hg * G) * D, q_bytes,
+                       &qfull);
+        }
+        ++items;
+      }
       bool valid = false;
       if (pg != kNoCand) {
         if (pg < 0 || pg >= num_pages) report(status, MSA_DEV_BAD_PAGE);
@@ -467,37 +462,36 @@ __global__ void __launch_bounds__(kPass1Threads + 32, 1) select_decode_pass1(
         s_item[s][0] = cur_b;
         s_item[s][1] = cur_c;
         s_item[s][2] = cur_gs;
-        mbar_expect_tx(&full[s], (uint32_t)(__popc(vb) + 1) * page_bytes);
+        mbar_expect_tx(&full[s], (uint32_t)__popc(vb) * page_bytes);
       }
       __syncwarp();
       if (valid)
         bulk_load_1d(st + (size_t)lane * pstride,
                      centroids + ((size_t)pg * hkv + (size_t)cur_gs * hg) * D, page_bytes, &full[s]);
-      if (lane == 0)
-        bulk_load_1d(st + (size_t)SC * pstride,
-                     qbar_all + ((size_t)cur_b * hkv + (size_t)cur_gs * hg) * D, page_bytes,
-                     &full[s]);
       if (++sub == KPL) {
         sub = 0;
-        it = claim();
+        it += gridDim.x;
+        if (it >= total_items) it = -1;
       }
       pg = it >= 0 ? fetch(it, sub) : kNoCand;
     }
     // every copy issued has landed before the CTA may end
     for (int m = n - NST < 0 ? 0 : n - NST; m < n; ++m)
       (void)mbar_wait(&full[m % NST], (uint32_t)(m / NST) & 1u);
+    if (items > 0) (void)mbar_wait(&qfull, (uint32_t)(items - 1) & 1u);
     return;
   }
 
   // ------------------------------- consumers -------------------------------
   const int my_g = tid / SC, my_k = tid - (tid / SC) * SC;
   const bool active = my_g < hg;
-  int n = 0;
+  int n = 0, items = 0;
 #pragma unroll 1
   for (;;) {
     uint64_t keys[KPL];
     int b = 0, c = 0, gs = 0;
     bool done = false;
+    const float* qbar = qbar2 + (items & 1) * hg * D;
 #pragma unroll
     for (int sub = 0; sub < KPL; ++sub, ++n) {
       const int s = n % NST;
@@ -512,13 +506,37 @@ __global__ void __launch_bounds__(kPass1Threads + 32, 1) select_decode_pass1(
       }
       c = s_item[s][1];
       gs = s_item[s][2];
+      if (sub == 0) {
+        // the item's qbar: each group's G heads summed left to right in fp32
+        if (!__all_sync(0xffffffffu, mbar_wait(&qfull, (uint32_t)items & 1u))) {
+          if (lane == 0) report(status, MSA_DEV_TIMEOUT);
+          return;
+        }
+        float* qb_w = qbar2 + (items & 1) * hg * D;
+        for (int x = tid; x < hg * D; x += kPass1Threads) {
+          const int gl = x / D, i = x - gl * D;
+          const T* src = qraw + (size_t)gl * G * D + i;
+          float a = to_f32(src[0]);
+          for (int h = 1; h < G; ++h) a = __fadd_rn(a, to_f32(src[(size_t)h * D]));
+          qb_w[x] = a;
+        }
+        // every consumer has its qbar (a bounded mbarrier wait, not bar.sync:
+        // a consumer that gave up on a wait must not leave the others stuck),
+        // and the raw rows may be replaced
+        mbar_arrive(&qready);
+        if (!__all_sync(0xffffffffu, mbar_wait(&qready, (uint32_t)items & 1u))) {
+          if (lane == 0) report(status, MSA_DEV_TIMEOUT);
+          return;
+        }
+        if (lane == 0) mbar_arrive(&qempty);
+        ++items;
+      }
       uint64_t key = 0ull;
       if (active && ((s_valid[s] >> my_k) & 1u)) {
         const unsigned char* st = smem_raw + (size_t)s * stage_bytes;
         const float4* cr = reinterpret_cast<const float4*>(st + (size_t)my_k * pstride +
                                                            (size_t)my_g * D * 4);
-        const float4* qb = reinterpret_cast<const float4*>(st + (size_t)SC * pstride +
-                                                           (size_t)my_g * D * 4);
+        const float4* qb = reinterpret_cast<const float4*>(qbar + (size_t)my_g * D);
         float acc = 0.f;
 #pragma unroll
         for (int x = 0; x < D / 4; ++x) {
@@ -877,24 +895,46 @@ cudaError_t select_rows(const msa_paged_kv_t* kv, const void* q, const int32_t* 
 
 bool select_rows_supported(int top_k) { return top_k - 1 <= 64; }
 
-// KV groups per pass-1 item: all of them up to 8 (one page copy of 4 KB for
-// d 128), else the largest divisor of hkv up to 8 (hkv itself if that is 1)
-static int pass1_groups(int hkv) {
-  if (hkv <= 8) return hkv;
-  for (int d = 8; d > 1; --d)
-    if (hkv % d == 0) return d;
-  return hkv;
+static int decode_nchunks(const msa_paged_kv_t* kv) {
+  return (kv->max_blocks_per_seq + kDecChunk - 1) / kDecChunk;
+}
+static int decode_kw(int top_k) { return top_k - 1 < kDecChunk ? (top_k - 1 < 1 ? 1 : top_k - 1) : kDecChunk; }
+
+static int device_sms() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+// KV groups per pass-1 item: the largest divisor of hkv up to 8 that still
+// makes about two items per SM (from the page-table width, an upper bound of
+// the chunks); a small batch gets fewer groups per item, hence more items
+// (one 1M-token sequence: 2 of 8 groups, 512 items instead of 128).
+static int pass1_groups(const msa_paged_kv_t* kv) {
+  const int hkv = kv->num_kv_heads;
+  const long chunks = (long)kv->batch * decode_nchunks(kv);
+  const long target = 2L * device_sms();
+  int smallest = hkv;
+  for (int d = hkv < 8 ? hkv : 8; d >= 1; --d) {
+    if (hkv % d) continue;
+    if (chunks * (hkv / d) >= target) return d;
+    if (d >= 2) smallest = d;
+  }
+  return hkv == 1 ? 1 : smallest;
 }
 static size_t pass1_smem(const msa_paged_kv_t* kv, int nst) {
-  return (size_t)nst * pass1_stage_bytes(pass1_groups(kv->num_kv_heads), kv->head_dim) +
-         (size_t)(2 * kv->batch + 1) * 4;
+  const int hg = pass1_groups(kv), D = kv->head_dim;
+  const size_t esz = kv->dtype == MSA_DTYPE_BF16 ? 2 : 4;
+  const size_t G = (size_t)(kv->num_q_heads / kv->num_kv_heads);
+  return (size_t)nst * pass1_stage_bytes(hg, D) + (size_t)hg * G * D * esz +
+         (size_t)2 * hg * D * 4 + (size_t)(2 * kv->batch + 1) * 4;
 }
 constexpr size_t kSmemLimit = 227 * 1024 - 1024;  // dynamic + static, per CTA
 // three stages where they fit (steps of up to 8 candidates), else two
 static int pass1_stages(const msa_paged_kv_t* kv) {
-  const int kpl = kDecChunk / pass1_sc(pass1_groups(kv->num_kv_heads));
-  const int nst = kpl <= 8 ? 3 : 2;
-  return pass1_smem(kv, nst) <= kSmemLimit ? nst : 0;
+  const int kpl = kDecChunk / pass1_sc(pass1_groups(kv));
+  if (kpl <= 8 && pass1_smem(kv, 3) <= kSmemLimit) return 3;
+  return pass1_smem(kv, 2) <= kSmemLimit ? 2 : 0;
 }
 
 // decode selection merges at most 32 * kMaxChunksPerLane chunk lists of
@@ -904,23 +944,13 @@ bool select_decode_supported(const msa_paged_kv_t* kv) {
          kv->num_kv_heads <= kPass1Threads / 2 && pass1_stages(kv) > 0;
 }
 
-static int decode_nchunks(const msa_paged_kv_t* kv) {
-  return (kv->max_blocks_per_seq + kDecChunk - 1) / kDecChunk;
-}
-static int decode_kw(int top_k) { return top_k - 1 < kDecChunk ? (top_k - 1 < 1 ? 1 : top_k - 1) : kDecChunk; }
-
-// workspace: chunk lists [batch][hkv][nchunks][kw] u64, qbar [batch][hkv][D] f32,
-// pass 1's work counter
+// workspace: chunk lists [batch][hkv][nchunks][kw] u64
 static size_t decode_lists_bytes(const msa_paged_kv_t* kv, int top_k) {
   const size_t b = (size_t)kv->batch * kv->num_kv_heads * decode_nchunks(kv) * decode_kw(top_k) * 8;
   return (b + 255) & ~(size_t)255;
 }
-static size_t decode_qbar_bytes(const msa_paged_kv_t* kv) {
-  const size_t b = (size_t)kv->batch * kv->num_kv_heads * kv->head_dim * 4;
-  return (b + 255) & ~(size_t)255;
-}
 size_t select_decode_ws(const msa_paged_kv_t* kv, int top_k) {
-  return decode_lists_bytes(kv, top_k) + decode_qbar_bytes(kv) + 256;
+  return decode_lists_bytes(kv, top_k) + 256;
 }
 
 // Resident pass-1 CTAs on the whole device, cached per (device, smem size).
@@ -944,31 +974,32 @@ static int pass1_slots(const void* fn, size_t smem) {
   return slots;
 }
 
-template <int D, int KPL, int NST>
-static cudaError_t launch_pass1(const msa_paged_kv_t* kv, const float* qbar, int kw, int nch,
-                                uint64_t* lists, unsigned int* counter, cudaStream_t st) {
+template <typename T, int D, int KPL, int NST>
+static cudaError_t launch_pass1(const msa_paged_kv_t* kv, const void* q, int kw, int nch,
+                                uint64_t* lists, cudaStream_t st) {
   const size_t smem = pass1_smem(kv, NST);
-  auto k1 = select_decode_pass1<D, KPL, NST>;
+  auto k1 = select_decode_pass1<T, D, KPL, NST>;
   cudaError_t e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  const int hg = pass1_groups(kv->num_kv_heads);
+  const int hg = pass1_groups(kv);
   const long upper = (long)kv->batch * nch * (kv->num_kv_heads / hg);
   const int grid = (int)std::max(1L, std::min<long>(upper, pass1_slots((const void*)k1, smem)));
-  return launch_pdl(k1, dim3(grid), dim3(kPass1Threads + 32), smem, st, (const float*)qbar,
+  return launch_pdl(k1, dim3(grid), dim3(kPass1Threads + 32), smem, st, (const T*)q,
                     (const float*)kv->centroids, (const int32_t*)kv->page_table,
-                    (const int32_t*)kv->seq_lens, kv->status_word, kv->batch, kv->num_kv_heads, hg,
-                    kv->block_size, kv->num_pages, kv->max_blocks_per_seq, kw, nch, lists, counter);
+                    (const int32_t*)kv->seq_lens, kv->status_word, kv->batch, kv->num_q_heads,
+                    kv->num_kv_heads, hg, kv->block_size, kv->num_pages, kv->max_blocks_per_seq, kw,
+                    nch, lists);
 }
 
-template <int D>
-static cudaError_t pass1_dispatch(const msa_paged_kv_t* kv, const float* qbar, int kw, int nch,
-                                  uint64_t* lists, unsigned int* counter, cudaStream_t st) {
-  switch (kDecChunk / pass1_sc(pass1_groups(kv->num_kv_heads))) {
-    case 2: return launch_pass1<D, 2, 3>(kv, qbar, kw, nch, lists, counter, st);
-    case 4: return launch_pass1<D, 4, 3>(kv, qbar, kw, nch, lists, counter, st);
-    case 8: return launch_pass1<D, 8, 3>(kv, qbar, kw, nch, lists, counter, st);
-    case 16: return launch_pass1<D, 16, 2>(kv, qbar, kw, nch, lists, counter, st);
-    default: return launch_pass1<D, 32, 2>(kv, qbar, kw, nch, lists, counter, st);
+template <typename T, int D, int NST>
+static cudaError_t pass1_dispatch_k(const msa_paged_kv_t* kv, const void* q, int kw, int nch,
+                                    uint64_t* lists, cudaStream_t st) {
+  switch (kDecChunk / pass1_sc(pass1_groups(kv))) {
+    case 2: return launch_pass1<T, D, 2, NST>(kv, q, kw, nch, lists, st);
+    case 4: return launch_pass1<T, D, 4, NST>(kv, q, kw, nch, lists, st);
+    case 8: return launch_pass1<T, D, 8, NST>(kv, q, kw, nch, lists, st);
+    case 16: return launch_pass1<T, D, 16, 2>(kv, q, kw, nch, lists, st);
+    default: return launch_pass1<T, D, 32, 2>(kv, q, kw, nch, lists, st);
   }
 }
 
@@ -977,12 +1008,8 @@ static cudaError_t launch_decode_sel(const msa_paged_kv_t* kv, const void* q, in
                                      int32_t* idx, float* score, void* ws, cudaStream_t st) {
   const int nch = decode_nchunks(kv), kw = decode_kw(top_k);
   uint64_t* lists = (uint64_t*)ws;
-  float* qbar = (float*)((char*)ws + decode_lists_bytes(kv, top_k));
-  unsigned int* counter = (unsigned int*)((char*)qbar + decode_qbar_bytes(kv));
-  cudaError_t e = launch_pdl(select_decode_qbar<T, D>, dim3(kv->num_kv_heads, kv->batch), dim3(D),
-                             0, st, (const T*)q, kv->num_q_heads, kv->num_kv_heads, qbar, counter);
-  if (e != cudaSuccess) return e;
-  e = pass1_dispatch<D>(kv, qbar, kw, nch, lists, counter, st);
+  cudaError_t e = pass1_stages(kv) == 3 ? pass1_dispatch_k<T, D, 3>(kv, q, kw, nch, lists, st)
+                                        : pass1_dispatch_k<T, D, 2>(kv, q, kw, nch, lists, st);
   if (e != cudaSuccess) return e;
   dim3 g2(kv->num_kv_heads, kv->batch);
   const int32_t* sl = kv->seq_lens;
