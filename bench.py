@@ -432,7 +432,7 @@ def run_decode(w, steps, warmup, world, flush_l2):
         raise RuntimeError(f"device status {status:#x}")
     return {"step_ms": per_step[0], "kernel_ms": k_ms, "clocks": clk.summary(),
             "e2e_ms": e2e_ms, "h2d": (hq_.numel() + hk.numel() + hv.numel()) * 2,
-            "d2h": hout.numel() * 2, "launches_per_step": 1 + 3 + 2}
+            "d2h": hout.numel() * 2, "launches_per_step": 1 + 2 + 2}
 
 
 def run_decode_steps(w, world):
@@ -533,7 +533,165 @@ def run_decode_steps(w, world):
     return {"step_ms": sum(step_ms) / S, "step_ms_first_last": [step_ms[0], step_ms[-1]],
             "kernel_ms": k_ms, "clocks": clk.summary(), "e2e_ms": e2e_ms,
             "h2d": (hq_[0].numel() + hk[0].numel() + hv[0].numel()) * 2,
-            "d2h": hout[0].numel() * 2, "launches_per_step": 1 + 3 + 2, "steps": S}
+            "d2h": hout[0].numel() * 2, "launches_per_step": 1 + 2 + 2, "steps": S}
+
+
+TOKEN_HEADS = 32      # indexer heads ("Sparse Attention + Linear Backbones", 5.3: 32 x 128)
+TOKEN_TOP_K = 2048    # kept positions per query (same section)
+
+
+def index_pages(w, p, lens, dev):
+    """Indexer keys of every sequence, one row per position, written into pages
+    of the cache's page table: [num_pages, block, d]."""
+    ki = torch.zeros(p.num_pages, w.block, w.d, dtype=w.torch_dtype, device=dev)
+    for b in range(w.batch):
+        L = lens[b]
+        nblk = -(-L // w.block)
+        rows = torch.zeros(nblk * w.block, w.d, dtype=w.torch_dtype, device=dev)
+        rows[:L] = workloads.indexer_keys(w, b, 0, L, dev)
+        ki[p.table[b, :nblk].long().to(dev)] = rows.view(nblk, w.block, w.d)
+    return ki
+
+
+def token_bytes(w, k):
+    """Algorithmic HBM bytes of one token-variant decode step: the indexer key of
+    every earlier position, the kept positions' K and V rows, q, out, the
+    indexer query, and the appended K/V row, its centroid and its indexer key."""
+    tot = 0
+    for b in range(w.batch):
+        L = w.ctx[b] + 1
+        tot += (L - 1) * w.d * 2 + min(k, L) * w.hkv * w.d * 2 * 2
+        tot += 2 * w.hq * w.d * 2 + TOKEN_HEADS * w.d * 2
+        tot += 2 * w.hkv * w.d * 2 + w.hkv * w.d * 4 + w.d * 2
+    return tot
+
+
+def run_tokens(w, steps, world):
+    """The token-granular variant on the paged-decode context: append one token
+    per sequence (with its indexer key), the indexer scores every earlier
+    position and keeps the top-K, then attention over the kept positions."""
+    import block_sparse_gqa_mean_b200 as msa
+    dev = torch.device("cuda")
+    cache = fill_decode_cache(w, dev)
+    after = [w.ctx[b] + 1 for b in range(w.batch)]
+    cache.seq_lens.copy_(torch.tensor(after, dtype=torch.int32))
+    p = workloads.paging(w)
+    ki = index_pages(w, p, after, dev)
+    kn, vn = workloads.new_tokens(w, 0, dev)
+    q = workloads.queries_decode(w, 0, dev).contiguous()
+    qi = workloads.indexer_queries(w, 0, TOKEN_HEADS, dev).contiguous()
+    # the appended token's indexer-key row: where it lives in the pages
+    last = torch.tensor([[int(p.table[b, (L - 1) // w.block]), (L - 1) % w.block]
+                         for b, L in enumerate(after)], dtype=torch.long, device=dev)
+    ki_new = torch.stack([ki[last[b, 0], last[b, 1]] for b in range(w.batch)]).contiguous()
+    cu = msa.cu_seqlens([1] * w.batch, dev)
+    tok = torch.empty(w.batch, TOKEN_TOP_K, dtype=torch.int32, device=dev)
+    out = torch.empty_like(q)
+    lse = torch.empty(w.batch, w.hq, dtype=torch.float32, device=dev)
+    ws = torch.empty(max(16, msa.workspace_size(msa.MSA_OP_SELECT_TOKENS, cache, w.batch, 1,
+                                                TOKEN_TOP_K)), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def do_append():
+        msa.build_block_cache(cache, kn, vn, cu, 1)
+        ki[last[:, 0], last[:, 1]] = ki_new          # the caller writes the indexer key
+
+    def do_select():
+        msa.select_tokens(cache, ki, qi, TOKEN_TOP_K, tok_idx=tok, workspace=ws)
+
+    def do_attn():
+        msa.sparse_attn_decode_tokens(cache, q, tok, out=out, lse=lse)
+
+    def step():
+        do_append()
+        do_select()
+        do_attn()
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    g_step = capture_graph(step)
+    g_ops = [capture_graph(f) for f in (do_append, do_select, do_attn)]
+    barrier(world)
+    torch.cuda.synchronize()
+    with Clocks(torch.cuda.current_device()) as clk:
+        step_ms = time_graph(g_step, steps)
+    k_ms = [time_graph(gg, steps) for gg in g_ops]
+    hq_, hqi = q.cpu().pin_memory(), qi.cpu().pin_memory()
+    hk, hv, hki = kn.cpu().pin_memory(), vn.cpu().pin_memory(), ki_new.cpu().pin_memory()
+    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    dq, dqi = torch.empty_like(q), torch.empty_like(qi)
+    dk, dv, dki = torch.empty_like(kn), torch.empty_like(vn), torch.empty_like(ki_new)
+    e2e = []
+    for _ in range(steps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for d_, h_ in ((dq, hq_), (dqi, hqi), (dk, hk), (dv, hv), (dki, hki)):
+            d_.copy_(h_, non_blocking=True)
+        msa.build_block_cache(cache, dk, dv, cu, 1)
+        ki[last[:, 0], last[:, 1]] = dki
+        msa.select_tokens(cache, ki, dqi, TOKEN_TOP_K, tok_idx=tok, workspace=ws)
+        msa.sparse_attn_decode_tokens(cache, dq, tok, out=out, lse=lse)
+        hout.copy_(out, non_blocking=True)
+        b.record(stream)
+        e2e.append((a, b))
+    torch.cuda.synchronize()
+    if cache.device_status() != 0:
+        raise RuntimeError(f"device status {cache.device_status():#x}")
+    h2d = sum(x.numel() * x.element_size() for x in (hq_, hqi, hk, hv, hki))
+    return {"step_ms": step_ms, "kernel_ms": k_ms, "clocks": clk.summary(),
+            "e2e_ms": sum(a.elapsed_time(b) for a, b in e2e) / steps, "h2d": h2d,
+            "d2h": hout.numel() * 2, "launches_per_step": 1 + 2 + 1}
+
+
+def tokens_block(w, args, world, pk):
+    """Block of the token-granular variant (decode form) on the paged-decode context."""
+    r = run_tokens(w, args.steps, world)
+    ms = max_over_ranks(r["step_ms"], world)
+    nbytes = token_bytes(w, TOKEN_TOP_K)
+    sel_b = sum((w.ctx[b]) * w.d * 2 + TOKEN_HEADS * w.d * 2 for b in range(w.batch))
+    att_b = sum(min(TOKEN_TOP_K, w.ctx[b] + 1) * w.hkv * w.d * 4 + 2 * w.hq * w.d * 2
+                for b in range(w.batch))
+    sel_ms, att_ms = r["kernel_ms"][1], r["kernel_ms"][2]
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"workload": w.name + " (token-granular indexer)", "value": w.batch * world / (ms * 1e-3),
+            "unit": "tokens/s", "ms_per_step": ms, "indexer_heads": TOKEN_HEADS,
+            "top_k_tokens": TOKEN_TOP_K,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / pk["hbm_gbs"], "traffic": None,
+                         "peak_source": f"{pk['source']} HBM copy",
+                         "scope": "whole decode step (append + indexer selection + attention)",
+                         "algorithmic_bytes_per_step": nbytes,
+                         "calls": {
+                             "select_tokens": {"bytes": sel_b, "ms": sel_ms,
+                                               "achieved_gbs": sel_b / (sel_ms * 1e-3) / 1e9},
+                             "sparse_attn_decode_tokens": {
+                                 "bytes": att_b, "ms": att_ms,
+                                 "achieved_gbs": att_b / (att_ms * 1e-3) / 1e9}}},
+            "kernels_ms": {"append": r["kernel_ms"][0], "select_tokens": sel_ms,
+                           "sparse_attn_decode_tokens": att_ms},
+            "e2e": {"value": w.batch * world / (r["e2e_ms"] * 1e-3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
+            "clocks": r["clocks"], "gpu_launches": r["launches_per_step"] * args.steps,
+            "l2": "step reads > 126 MB L2, no flush"}
+
+
+def oracle_tokens_sample(w, device="cpu"):
+    """Oracle of the token variant on sequence 0's decode step (inputs drawn on
+    `device`, outside the timed region). Returns (sequences, seconds, threads)."""
+    import oracle
+    L = w.ctx[0] + 1
+    K = workloads.keys(w, 0, 0, L, device).cpu()
+    V = workloads.values(w, 0, 0, L, device).cpu()
+    KI = workloads.indexer_keys(w, 0, 0, L, device).cpu()
+    Q = workloads.queries_decode(w, 0, seqs=[0])
+    QI = workloads.indexer_queries(w, 0, TOKEN_HEADS)[:1]
+    pos = np.array([L - 1])
+    t = time.perf_counter()
+    S = oracle.token_scores(QI, KI, pos)
+    idx, _ = oracle.token_select(S, pos, TOKEN_TOP_K)
+    oracle.attend_tokens(Q, K, V, pos, idx, w.softmax_scale)
+    return 1, time.perf_counter() - t, 1
 
 
 def run_tiny(w, steps, world):
@@ -661,7 +819,7 @@ def main():
     ap.add_argument("--workload", default="prefill_bf16", choices=list(workloads.ALL))
     ap.add_argument("--no-decode", action="store_true",
                     help="skip the blocks of the other workloads")
-    ap.add_argument("--blocks", default="decode,decode_1m,varlen,tiny",
+    ap.add_argument("--blocks", default="decode,decode_1m,varlen,tiny,tokens",
                     help="workload blocks measured after the prefill headline")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--oracle-rows", type=int, default=256)
@@ -811,6 +969,17 @@ def extra_blocks(args, world, pk):
         elif key == "tiny":
             w = workloads.tiny_f32()
             out[key] = tiny_block(w, args, world, pk)
+        elif key == "tokens":
+            w = workloads.paged_decode_bf16()
+            out[key] = tokens_block(w, args, world, pk)
+            if not args.no_cpu_baseline and world == 1:
+                n, secs, thr = oracle_tokens_sample(w, "cuda")
+                out[key]["cpu_baseline"] = {
+                    "value": n / secs, "unit": "tokens/s", "cores": thr, "kind": "oracle",
+                    "sample": f"sequence 0's decode step ({w.ctx[0] + 1} positions): indexer "
+                              f"scores, top-{TOKEN_TOP_K}, attention; numpy fp64"}
+            out[key]["config"] = workload_config(w)
+            continue
         else:
             raise SystemExit(f"unknown block {key}")
         if not args.no_cpu_baseline and world == 1:

@@ -17,7 +17,7 @@
 // to 16 rows, keeps an online softmax per row, and the warps are merged in
 // shared memory. The CTA writes its normalised partial (o, lse); a second
 // kernel merges the splits by log-sum-exp and rounds to bf16.
-#include "tma.cuh"
+#include "mma_sync.cuh"
 
 namespace msa {
 
@@ -25,41 +25,7 @@ namespace {
 
 constexpr int kD = 128;
 constexpr float kLog2e = 1.4426950408889634f;
-
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&v);
-}
-
-__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
-                                               uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
-                                        uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(addr));
-}
-
-__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
-                                          uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-               : "r"(addr));
-}
-
-// Address of the 16-byte chunk (row r, chunk c in 0..15 over 128 columns) of
-// a swizzled tile made of two [rows][64] halves.
-__device__ __forceinline__ uint32_t tile_chunk(uint32_t tile, int rows, int r, int c) {
-  return tile + (uint32_t)(c >> 3) * (uint32_t)rows * 128u + sw128_offset(r, c & 7);
-}
-
+using namespace warpmma;
 }  // namespace
 
 template <int B>
@@ -245,10 +211,10 @@ __global__ void __launch_bounds__(128) decode_splitk_kernel(
 #pragma unroll
     for (int kk = 0; kk < NT / 2; ++kk) {
       uint32_t pa[4];
-      pa[0] = pack_bf16(s[2 * kk][0], s[2 * kk][1]);
-      pa[1] = pack_bf16(s[2 * kk][2], s[2 * kk][3]);
-      pa[2] = pack_bf16(s[2 * kk + 1][0], s[2 * kk + 1][1]);
-      pa[3] = pack_bf16(s[2 * kk + 1][2], s[2 * kk + 1][3]);
+      pa[0] = pack_bf16x2(s[2 * kk][0], s[2 * kk][1]);
+      pa[1] = pack_bf16x2(s[2 * kk][2], s[2 * kk][3]);
+      pa[2] = pack_bf16x2(s[2 * kk + 1][0], s[2 * kk + 1][1]);
+      pa[3] = pack_bf16x2(s[2 * kk + 1][2], s[2 * kk + 1][3]);
       const int kb = warp * KW + 16 * kk;
       const int key = kb + (lane & 7) + 8 * ((lane >> 3) & 1);
 #pragma unroll

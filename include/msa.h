@@ -299,8 +299,9 @@ msa_status_t msa_sparse_attn_decode_noalloc(const msa_paged_kv_t* kv, const void
  * kept; attention over those positions). The page leaves the indexer's form
  * open; it is read here like the block score: for the query at t = seq_lens[b]-1
  *   s(u) = sum_h qi[b][h] . ki[u]        (u < t; fp32: the heads summed left to
- *                                         right, then one fma chain in
- *                                         coordinate order),
+ *                                         right, an fma chain over each
+ *                                         16-byte chunk of the key, then the
+ *                                         chunks' sums added pairwise),
  *   kept = {t} plus the top_k-1 best u < t (all of them when t < top_k),
  *          ties to the lower position.
  *
