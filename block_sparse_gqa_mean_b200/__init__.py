@@ -35,7 +35,9 @@ MSA_DEV_BAD_PAGE, MSA_DEV_BAD_LENGTH, MSA_DEV_BAD_INDEX, MSA_DEV_TIMEOUT = 1, 2,
 EXPORTS = ("msa_build_block_cache", "msa_select_topk", "msa_sparse_attn_prefill",
            "msa_sparse_attn_decode", "msa_sparse_attn_prefill_gated",
            "msa_sparse_attn_decode_gated", "msa_sparse_attn_decode_noalloc", "msa_workspace_size",
-           "msa_status_string", "msa_version", "msa_select_tokens", "msa_sparse_attn_decode_tokens")
+           "msa_status_string", "msa_version", "msa_select_tokens", "msa_sparse_attn_decode_tokens",
+           "msa_select_topk_range", "msa_select_merge", "msa_sparse_attn_decode_range",
+           "msa_lse_merge")
 
 
 class MsaError(RuntimeError):
@@ -89,6 +91,11 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                                                  SZ, P]
     lib.msa_select_tokens.argtypes = [KV, P, P, I32, I32, P, P, SZ, P]
     lib.msa_sparse_attn_decode_tokens.argtypes = [KV, P, P, I32, ctypes.c_float, P, P, P]
+    lib.msa_select_topk_range.argtypes = [KV, P, I32, I32, I32, P, P, SZ, P]
+    lib.msa_select_merge.argtypes = [KV, P, I32, I32, P, P, P]
+    lib.msa_sparse_attn_decode_range.argtypes = [KV, P, P, I32, I32, I32, ctypes.c_float, P, P, P,
+                                                 SZ, P]
+    lib.msa_lse_merge.argtypes = [P, P, I32, I32, I32, I32, P, P, P]
     lib.msa_workspace_size.argtypes = [ctypes.c_int, KV, I32, I32, I32]
     lib.msa_workspace_size.restype = SZ
     lib.msa_status_string.argtypes = [ctypes.c_int]
@@ -97,7 +104,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     for name in ("msa_build_block_cache", "msa_select_topk", "msa_sparse_attn_prefill",
                  "msa_sparse_attn_decode", "msa_sparse_attn_prefill_gated",
                  "msa_sparse_attn_decode_gated", "msa_sparse_attn_decode_noalloc",
-                 "msa_select_tokens", "msa_sparse_attn_decode_tokens"):
+                 "msa_select_tokens", "msa_sparse_attn_decode_tokens", "msa_select_topk_range",
+                 "msa_select_merge", "msa_sparse_attn_decode_range", "msa_lse_merge"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -378,6 +386,107 @@ def sparse_attn_decode_tokens(cache: PagedKVCache, q: torch.Tensor, tok_idx: tor
                                              scale, _ptr(out), _ptr(lse), _stream(stream)),
            "msa_sparse_attn_decode_tokens")
     return out, lse
+
+
+# ---------------------------------------------------------------------------
+# context-sharded decode (blocks of every sequence split over ranks by range)
+# ---------------------------------------------------------------------------
+def select_topk_range(cache: PagedKVCache, q: torch.Tensor, top_k: int, block_lo: int,
+                      block_hi: int, cand_keys: Optional[torch.Tensor] = None,
+                      workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """This rank's best top_k-1 candidates among blocks [block_lo, block_hi) of
+    every sequence's decode row: [batch, Hkv, top_k-1] selection keys (int64
+    bit patterns of the library's unsigned keys, descending, 0 padded)."""
+    lib = load_library()
+    _require_cuda(q, cand_keys)
+    if cand_keys is None:
+        cand_keys = torch.zeros(q.shape[0], cache.num_kv_heads, max(top_k - 1, 1),
+                                dtype=torch.int64, device=q.device)
+    ws, ws_bytes = _workspace(MSA_OP_SELECT, cache, q.shape[0], 1, top_k, workspace)
+    kv = cache.struct()
+    _check(lib.msa_select_topk_range(ctypes.byref(kv), _ptr(q), int(block_lo), int(block_hi),
+                                     top_k, _ptr(cand_keys), _ptr(ws), ws_bytes, _stream(stream)),
+           "msa_select_topk_range")
+    return cand_keys
+
+
+def select_merge(cache: PagedKVCache, cand_keys: torch.Tensor, top_k: int,
+                 block_idx: Optional[torch.Tensor] = None, want_scores: bool = False,
+                 stream=None):
+    """Global selection from the ranks' gathered candidate keys
+    [num_lists, batch, Hkv, top_k-1]: the block lists msa_select_topk gives for
+    the unsharded sequences."""
+    lib = load_library()
+    _require_cuda(cand_keys, block_idx)
+    nl, batch = cand_keys.shape[0], cand_keys.shape[1]
+    if block_idx is None:
+        block_idx = torch.empty(batch, cache.num_kv_heads, top_k, dtype=torch.int32,
+                                device=cand_keys.device)
+    score = (torch.empty(batch, cache.num_kv_heads, top_k, dtype=torch.float32,
+                         device=cand_keys.device) if want_scores else None)
+    kv = cache.struct()
+    _check(lib.msa_select_merge(ctypes.byref(kv), _ptr(cand_keys), nl, top_k, _ptr(block_idx),
+                                _ptr(score), _stream(stream)), "msa_select_merge")
+    return block_idx, score
+
+
+def sparse_attn_decode_range(cache: PagedKVCache, q: torch.Tensor, block_idx: torch.Tensor,
+                             block_lo: int, block_hi: int, softmax_scale: Optional[float] = None,
+                             workspace: Optional[torch.Tensor] = None, stream=None):
+    """This rank's attention partial over the selected blocks in [block_lo,
+    block_hi): (o_part [batch, Hq, d] fp32 normalised, lse_part [batch, Hq])."""
+    lib = load_library()
+    _require_cuda(q, block_idx)
+    top_k = block_idx.shape[-1]
+    scale = 1.0 / math.sqrt(cache.head_dim) if softmax_scale is None else softmax_scale
+    o_part = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    lse_part = torch.empty(q.shape[0], q.shape[1], dtype=torch.float32, device=q.device)
+    ws, ws_bytes = _workspace(MSA_OP_DECODE, cache, q.shape[0], 1, top_k, workspace)
+    kv = cache.struct()
+    _check(lib.msa_sparse_attn_decode_range(ctypes.byref(kv), _ptr(q), _ptr(block_idx), top_k,
+                                            int(block_lo), int(block_hi), scale, _ptr(o_part),
+                                            _ptr(lse_part), _ptr(ws), ws_bytes, _stream(stream)),
+           "msa_sparse_attn_decode_range")
+    return o_part, lse_part
+
+
+def lse_merge(o_parts: torch.Tensor, lse_parts: torch.Tensor, dtype=torch.bfloat16, stream=None):
+    """Log-sum-exp merge of partials [P, batch, Hq, d] / [P, batch, Hq] ->
+    (out [batch, Hq, d] in dtype, lse [batch, Hq])."""
+    lib = load_library()
+    _require_cuda(o_parts, lse_parts)
+    P, d = o_parts.shape[0], o_parts.shape[-1]
+    rows = o_parts[0].numel() // d
+    out = torch.empty(o_parts.shape[1:], dtype=dtype, device=o_parts.device)
+    lse = torch.empty(lse_parts.shape[1:], dtype=torch.float32, device=o_parts.device)
+    dt = MSA_DTYPE_BF16 if dtype == torch.bfloat16 else MSA_DTYPE_F32
+    _check(lib.msa_lse_merge(_ptr(o_parts), _ptr(lse_parts), P, rows, d, dt, _ptr(out), _ptr(lse),
+                             _stream(stream)), "msa_lse_merge")
+    return out, lse
+
+
+def sharded_decode(cache: PagedKVCache, q: torch.Tensor, top_k: int, block_lo: int,
+                   block_hi: int, group=None, ops=None):
+    """One decode step of context-sharded sequences: this rank holds blocks
+    [block_lo, block_hi) of every sequence. Two all-gathers over the process
+    group (the ranks' candidate keys; the ranks' attention partials) surround
+    the library calls; every rank returns the same (out, lse, block_idx).
+    `ops` replaces the four per-rank calls (tests of the exchange on CPU)."""
+    import torch.distributed as dist
+    ops = ops or {"select": select_topk_range, "merge": select_merge,
+                  "attend": sparse_attn_decode_range, "combine": lse_merge}
+    world = dist.get_world_size(group)
+
+    def gather(x):  # [world, ...] in rank order
+        parts = [torch.empty_like(x) for _ in range(world)]
+        dist.all_gather(parts, x.contiguous(), group=group)
+        return torch.stack(parts)
+
+    keys = ops["select"](cache, q, top_k, block_lo, block_hi)
+    block_idx, _ = ops["merge"](cache, gather(keys), top_k)
+    o_part, lse_part = ops["attend"](cache, q, block_idx, block_lo, block_hi)
+    out, lse = ops["combine"](gather(o_part), gather(lse_part), dtype=q.dtype)
+    return out, lse, block_idx
 
 
 def cu_seqlens(lengths, device="cuda") -> torch.Tensor:

@@ -34,7 +34,8 @@ __global__ void __launch_bounds__(128) decode_splitk_kernel(
     const bf16* __restrict__ q, const int32_t* __restrict__ block_idx,
     const int32_t* __restrict__ page_table, const int32_t* __restrict__ seq_lens, uint32_t* status,
     int top_k, int hq, int hkv, int num_pages, int max_blocks, float scale_log2, int splits,
-    int per_split, float* __restrict__ ws_o, float* __restrict__ ws_lse) {
+    int per_split, int block_lo, int block_hi, float* __restrict__ ws_o,
+    float* __restrict__ ws_lse) {
   constexpr int NST = 2;                 // pipeline stages
   constexpr int TILE = B * kD * 2;       // bytes of one K (or V) tile
   constexpr int KW = B / 4;              // keys per warp per block
@@ -76,6 +77,8 @@ __global__ void __launch_bounds__(128) decode_splitk_kernel(
       j = sel[base + tid];
       // a block repeated in the adjacent slot (rows are ascending) counts once
       if (j >= 0 && s0 + base + tid > 0 && sel[base + tid - 1] == j) j = -1;
+      // context-sharded decode: blocks outside this rank's range are another's
+      if (j >= 0 && j <= t / B && (j < block_lo || j >= block_hi)) j = -1;
       if (j >= 0) {
         if (j > t / B) {
           report(status, MSA_DEV_BAD_INDEX);
@@ -331,9 +334,10 @@ static size_t decode_smem(int B) {
   return (stages > red ? stages : red) + 1024;
 }
 
-cudaError_t decode_splitk(const msa_paged_kv_t* kv, const void* q, const int32_t* idx, int top_k,
-                          float scale, void* out, float* lse, void* ws, int num_sms, gate_t gate,
-                          cudaStream_t st) {
+static cudaError_t decode_splitk_any(const msa_paged_kv_t* kv, const void* q, const int32_t* idx,
+                                     int top_k, float scale, void* out, bool f32_out, float* lse,
+                                     void* ws, int num_sms, gate_t gate, int lo, int hi,
+                                     cudaStream_t st) {
   const int B = kv->block_size;
   const int splits = decode_splits(kv, top_k, num_sms);
   const int per = (top_k + splits - 1) / splits;
@@ -356,7 +360,7 @@ cudaError_t decode_splitk(const msa_paged_kv_t* kv, const void* q, const int32_t
     e = launch_pdl(decode_splitk_kernel<64>, grid, dim3(128), smem, st, tk, tv, (const bf16*)q,
                    idx, (const int32_t*)kv->page_table, (const int32_t*)kv->seq_lens,
                    kv->status_word, top_k, kv->num_q_heads, kv->num_kv_heads, kv->num_pages,
-                   kv->max_blocks_per_seq, sl2, splits, per, ws_o, ws_lse);
+                   kv->max_blocks_per_seq, sl2, splits, per, lo, hi, ws_o, ws_lse);
   } else {
     e = cudaFuncSetAttribute(decode_splitk_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem);
@@ -364,11 +368,67 @@ cudaError_t decode_splitk(const msa_paged_kv_t* kv, const void* q, const int32_t
     e = launch_pdl(decode_splitk_kernel<128>, grid, dim3(128), smem, st, tk, tv, (const bf16*)q,
                    idx, (const int32_t*)kv->page_table, (const int32_t*)kv->seq_lens,
                    kv->status_word, top_k, kv->num_q_heads, kv->num_kv_heads, kv->num_pages,
-                   kv->max_blocks_per_seq, sl2, splits, per, ws_o, ws_lse);
+                   kv->max_blocks_per_seq, sl2, splits, per, lo, hi, ws_o, ws_lse);
   }
   if (e != cudaSuccess) return e;
+  if (f32_out)
+    return launch_pdl(decode_combine_kernel<float>, dim3(kv->batch * kv->num_q_heads), dim3(128),
+                      0, st, (const float*)ws_o, (const float*)ws_lse, splits, (float*)out, lse,
+                      gate);
   return launch_pdl(decode_combine_kernel<bf16>, dim3(kv->batch * kv->num_q_heads), dim3(128), 0,
                     st, (const float*)ws_o, (const float*)ws_lse, splits, (bf16*)out, lse, gate);
+}
+
+cudaError_t decode_splitk(const msa_paged_kv_t* kv, const void* q, const int32_t* idx, int top_k,
+                          float scale, void* out, float* lse, void* ws, int num_sms, gate_t gate,
+                          cudaStream_t st) {
+  return decode_splitk_any(kv, q, idx, top_k, scale, out, false, lse, ws, num_sms, gate, 0,
+                           0x7fffffff, st);
+}
+
+// Context-sharded decode: this rank's normalised fp32 partial and its lse over
+// the selected blocks in [lo, hi).
+cudaError_t decode_splitk_range(const msa_paged_kv_t* kv, const void* q, const int32_t* idx,
+                                int top_k, float scale, float* o_part, float* lse_part, void* ws,
+                                int num_sms, int lo, int hi, cudaStream_t st) {
+  return decode_splitk_any(kv, q, idx, top_k, scale, o_part, true, lse_part, ws, num_sms, gate_t{},
+                           lo, hi, st);
+}
+
+// Log-sum-exp merge of num_parts normalised partials: o_parts [num_parts][rows][D]
+// fp32, lse_parts [num_parts][rows] (natural log, -inf: no keys) -> out [rows][D]
+// in T, lse [rows] (may be null).
+template <typename T>
+__global__ void __launch_bounds__(128) lse_merge_kernel(const float* __restrict__ o_parts,
+                                                        const float* __restrict__ lse_parts,
+                                                        int num_parts, int rows, int D,
+                                                        T* __restrict__ out,
+                                                        float* __restrict__ lse) {
+  pdl_wait();
+  const size_t r = blockIdx.x;
+  float M = -INFINITY;
+  for (int p = 0; p < num_parts; ++p) M = fmaxf(M, lse_parts[(size_t)p * rows + r]);
+  float w = 0.f;
+  if (M != -INFINITY)
+    for (int p = 0; p < num_parts; ++p) w += expf(lse_parts[(size_t)p * rows + r] - M);
+  for (int i = threadIdx.x; i < D; i += blockDim.x) {
+    float acc = 0.f;
+    if (M != -INFINITY)
+      for (int p = 0; p < num_parts; ++p)
+        acc += expf(lse_parts[(size_t)p * rows + r] - M) * o_parts[((size_t)p * rows + r) * D + i];
+    out[r * D + i] = from_f32<T>(w > 0.f ? acc / w : 0.f);
+  }
+  if (lse && threadIdx.x == 0) lse[r] = w > 0.f ? M + logf(w) : -INFINITY;
+  pdl_release();
+}
+
+cudaError_t lse_merge(const float* o_parts, const float* lse_parts, int num_parts, int rows, int D,
+                      bool bf16_out, void* out, float* lse, cudaStream_t st) {
+  if (bf16_out)
+    return launch_pdl(lse_merge_kernel<bf16>, dim3(rows), dim3(128), 0, st, o_parts, lse_parts,
+                      num_parts, rows, D, (bf16*)out, lse);
+  return launch_pdl(lse_merge_kernel<float>, dim3(rows), dim3(128), 0, st, o_parts, lse_parts,
+                    num_parts, rows, D, (float*)out, lse);
 }
 
 }  // namespace msa

@@ -28,6 +28,13 @@ cudaError_t select_tokens(const msa_paged_kv_t*, const void*, const void*, int, 
                           cudaStream_t);
 cudaError_t attn_tokens(const msa_paged_kv_t*, const void*, const int32_t*, int, float, void*,
                         float*, cudaStream_t);
+cudaError_t select_decode_range(const msa_paged_kv_t*, const void*, int, int, int, uint64_t*, void*,
+                                cudaStream_t);
+cudaError_t select_merge_lists(const msa_paged_kv_t*, const uint64_t*, int, int, int32_t*, float*,
+                               cudaStream_t);
+cudaError_t decode_splitk_range(const msa_paged_kv_t*, const void*, const int32_t*, int, float,
+                                float*, float*, void*, int, int, int, cudaStream_t);
+cudaError_t lse_merge(const float*, const float*, int, int, int, bool, void*, float*, cudaStream_t);
 bool prefill_tc_supported(const msa_paged_kv_t*);
 size_t prefill_ws(const msa_paged_kv_t*, int max_rows, int top_k);
 cudaError_t prefill_tc(const msa_paged_kv_t*, const void*, const int32_t*, int, const int32_t*,
@@ -326,6 +333,76 @@ msa_status_t msa_sparse_attn_decode_tokens(const msa_paged_kv_t* kv, const void*
     return MSA_ERR_INVALID_ARG;
   return msa::from_cuda(msa::attn_tokens(kv, q, tok_idx, top_k, softmax_scale, out, lse,
                                          (cudaStream_t)stream));
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// context-sharded decode
+// ---------------------------------------------------------------------------
+extern "C" {
+
+msa_status_t msa_select_topk_range(const msa_paged_kv_t* kv, const void* q, int32_t block_lo,
+                                   int32_t block_hi, int32_t top_k, uint64_t* cand_keys,
+                                   void* workspace, size_t workspace_bytes, msa_stream_t stream) {
+  msa_status_t s = msa::check_kv(kv);
+  if (s != MSA_OK) return s;
+  if (top_k < 1 || top_k - 1 > 64) return MSA_ERR_UNSUPPORTED;
+  if (!msa::select_decode_supported(kv)) return MSA_ERR_UNSUPPORTED;
+  if (!q || !msa::aligned(q, 16) || block_lo < 0 || block_hi < block_lo ||
+      (top_k > 1 && (!cand_keys || !msa::aligned(cand_keys, 8))))
+    return MSA_ERR_INVALID_ARG;
+  const size_t need = msa::select_decode_ws(kv, top_k);
+  if (workspace_bytes < need || !workspace || !msa::aligned(workspace, 16))
+    return MSA_ERR_WORKSPACE;
+  return msa::from_cuda(msa::select_decode_range(kv, q, top_k, block_lo, block_hi, cand_keys,
+                                                 workspace, (cudaStream_t)stream));
+}
+
+msa_status_t msa_select_merge(const msa_paged_kv_t* kv, const uint64_t* cand_keys,
+                              int32_t num_lists, int32_t top_k, int32_t* block_idx,
+                              float* block_score, msa_stream_t stream) {
+  msa_status_t s = msa::check_kv(kv);
+  if (s != MSA_OK) return s;
+  if (top_k < 1 || top_k - 1 > 64) return MSA_ERR_UNSUPPORTED;
+  if (num_lists < 1 || !block_idx || !msa::aligned(block_idx, 4) ||
+      (block_score && !msa::aligned(block_score, 4)) ||
+      (top_k > 1 && (!cand_keys || !msa::aligned(cand_keys, 8))))
+    return MSA_ERR_INVALID_ARG;
+  return msa::from_cuda(msa::select_merge_lists(kv, cand_keys, num_lists, top_k, block_idx,
+                                                block_score, (cudaStream_t)stream));
+}
+
+msa_status_t msa_sparse_attn_decode_range(const msa_paged_kv_t* kv, const void* q,
+                                          const int32_t* block_idx, int32_t top_k,
+                                          int32_t block_lo, int32_t block_hi, float softmax_scale,
+                                          float* o_part, float* lse_part, void* workspace,
+                                          size_t workspace_bytes, msa_stream_t stream) {
+  msa_status_t s = msa::check_decode_args(kv, q, block_idx, top_k, softmax_scale, o_part, lse_part);
+  if (s != MSA_OK) return s;
+  if (!msa::use_decode_splitk(kv)) return MSA_ERR_UNSUPPORTED;
+  if (!lse_part || block_lo < 0 || block_hi < block_lo) return MSA_ERR_INVALID_ARG;
+  const int sms = msa::num_sms();
+  const size_t need = msa::decode_ws(kv, top_k, sms);
+  if (workspace_bytes < need || !workspace || !msa::aligned(workspace, 16))
+    return MSA_ERR_WORKSPACE;
+  return msa::from_cuda(msa::decode_splitk_range(kv, q, block_idx, top_k, softmax_scale, o_part,
+                                                 lse_part, workspace, sms, block_lo, block_hi,
+                                                 (cudaStream_t)stream));
+}
+
+msa_status_t msa_lse_merge(const float* o_parts, const float* lse_parts, int32_t num_parts,
+                           int32_t rows, int32_t head_dim, int32_t out_dtype, void* out,
+                           float* lse, msa_stream_t stream) {
+  if (num_parts < 1 || rows < 0 || head_dim < 1) return MSA_ERR_INVALID_ARG;
+  if (out_dtype != MSA_DTYPE_BF16 && out_dtype != MSA_DTYPE_F32) return MSA_ERR_UNSUPPORTED;
+  if (rows == 0) return MSA_OK;
+  if (!o_parts || !lse_parts || !out || !msa::aligned(o_parts, 4) || !msa::aligned(lse_parts, 4) ||
+      !msa::aligned(out, 4) || (lse && !msa::aligned(lse, 4)))
+    return MSA_ERR_INVALID_ARG;
+  return msa::from_cuda(msa::lse_merge(o_parts, lse_parts, num_parts, rows, head_dim,
+                                       out_dtype == MSA_DTYPE_BF16, out, lse,
+                                       (cudaStream_t)stream));
 }
 
 }  // extern "C"

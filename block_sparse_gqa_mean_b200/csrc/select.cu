@@ -327,7 +327,7 @@ __global__ void __launch_bounds__(kPass1Threads + 32, 1) select_decode_pass1(
     const T* __restrict__ q, const float* __restrict__ centroids,
     const int32_t* __restrict__ page_table, const int32_t* __restrict__ seq_lens, uint32_t* status,
     int batch, int hq, int hkv, int hg, int B, int num_pages, int max_blocks, int kw, int nchunks,
-    uint64_t* __restrict__ ws) {
+    int cand_lo, int cand_hi, uint64_t* __restrict__ ws) {
   constexpr int SC = kDecChunk / KPL;         // candidates per step = lanes per group
   constexpr int NCW = kPass1Threads / 32;     // consumer warps
   constexpr int NW = NCW + 1;
@@ -374,7 +374,8 @@ __global__ void __launch_bounds__(kPass1Threads + 32, 1) select_decode_pass1(
       if (L < 1 || L > max_blocks * B) {
         if (blockIdx.x == 0) report(status, MSA_DEV_BAD_LENGTH);
       } else {
-        nc = (L - 1) / B;
+        // candidates: complete past blocks in [cand_lo, cand_hi)
+        nc = max(0, min((L - 1) / B, cand_hi) - cand_lo);
         n = (nc + kDecChunk - 1) / kDecChunk * hsplit;
       }
       ncs[b] = nc;
@@ -416,7 +417,8 @@ __global__ void __launch_bounds__(kPass1Threads + 32, 1) select_decode_pass1(
       cur_c = r / hsplit;
       cur_gs = r - cur_c * hsplit;
       const int j = cur_c * kDecChunk + sub * SC + lane;
-      return (lane < SC && j < ncs[lo]) ? page_table[(size_t)lo * max_blocks + j] : kNoCand;
+      return (lane < SC && j < ncs[lo]) ? page_table[(size_t)lo * max_blocks + cand_lo + j]
+                                        : kNoCand;
     };
     int it = (int)blockIdx.x < total_items ? (int)blockIdx.x : -1, sub = 0;
     int pg = it >= 0 ? fetch(it, 0) : kNoCand;
@@ -547,7 +549,7 @@ __global__ void __launch_bounds__(kPass1Threads + 32, 1) select_decode_pass1(
           acc = __fmaf_rn(qv.z, cv.z, acc);
           acc = __fmaf_rn(qv.w, cv.w, acc);
         }
-        key = sel_key(acc, c * kDecChunk + sub * SC + my_k);
+        key = sel_key(acc, cand_lo + c * kDecChunk + sub * SC + my_k);
       }
       keys[sub] = key;
       __syncwarp();
@@ -647,11 +649,18 @@ __device__ __forceinline__ void warp_merge_top(uint64_t (&a)[NK], const uint64_t
 // into its running top 32·NK, warp 0 merges the four warps' lists, and a
 // bitonic sort on the block index (NK elements per lane) gives the ascending
 // output.
+// The same kernel merges (a) the chunk lists of one sequence's candidates in
+// [cand_lo, cand_hi) (nlists = 0: one list per chunk of 64 candidates, list c
+// of (b, g) at ws + ((b * hkv + g) * nchunks + c) * kw), or (b) nlists lists
+// gathered from the ranks of a context-sharded decode (list c of (b, g) at
+// ws + ((c * batch + b) * hkv + g) * kw). With keys_out it writes the best
+// min(k-1, candidates) keys of each (b, g), descending, 0 padded to top_k - 1,
+// instead of the ascending block list.
 template <int NK, int LG>
 __global__ void __launch_bounds__(128) select_decode_merge(
-    const uint64_t* __restrict__ ws, const int32_t* __restrict__ seq_lens, int hkv, int B,
-    int max_blocks, int kw, int nchunks, int top_k, int32_t* __restrict__ idx,
-    float* __restrict__ score) {
+    const uint64_t* __restrict__ ws, const int32_t* __restrict__ seq_lens, int batch, int hkv,
+    int B, int max_blocks, int kw, int nchunks, int top_k, int nlists, int cand_lo, int cand_hi,
+    int32_t* __restrict__ idx, float* __restrict__ score, uint64_t* __restrict__ keys_out) {
   __shared__ uint64_t part[4][32 * NK];
   pdl_wait();
   const int g = blockIdx.x, b = blockIdx.y;
@@ -660,9 +669,12 @@ __global__ void __launch_bounds__(128) select_decode_merge(
   const size_t outo = ((size_t)b * hkv + g) * top_k;
   if (L < 1 || L > max_blocks * B) return;  // reported by pass 1
   const int own = (L - 1) / B;
-  const int keep = min(top_k - 1, own);
-  const int nch = (own + kDecChunk - 1) / kDecChunk;
-  const uint64_t* src = ws + ((size_t)b * hkv + g) * nchunks * kw;
+  const int ncand = max(0, min(own, cand_hi) - cand_lo);
+  const int keep = min(top_k - 1, ncand);
+  const int nch = nlists > 0 ? nlists : (ncand + kDecChunk - 1) / kDecChunk;
+  const uint64_t* src = nlists > 0 ? ws + ((size_t)b * hkv + g) * kw
+                                   : ws + ((size_t)b * hkv + g) * nchunks * kw;
+  const size_t lstride = nlists > 0 ? (size_t)batch * hkv * kw : (size_t)kw;
   uint64_t acc[NK];
 #pragma unroll
   for (int r = 0; r < NK; ++r) acc[r] = 0ull;
@@ -674,7 +686,7 @@ __global__ void __launch_bounds__(128) select_decode_merge(
 #pragma unroll
       for (int r = 0; r < NK; ++r) {
         const int i = lane + 32 * r;
-        l[u][r] = (c < nch && i < kw) ? src[(size_t)c * kw + i] : 0ull;
+        l[u][r] = (c < nch && i < kw) ? src[(size_t)c * lstride + i] : 0ull;
       }
     }
 #pragma unroll
@@ -699,6 +711,16 @@ __global__ void __launch_bounds__(128) select_decode_merge(
   warp_merge_top<NK>(m0, m1, lane);
   warp_merge_top<NK>(m2, m3, lane);
   warp_merge_top<NK>(m0, m2, lane);
+  if (keys_out) {  // the best keys themselves, descending
+    uint64_t* ko = keys_out + ((size_t)b * hkv + g) * (top_k - 1);
+#pragma unroll
+    for (int r = 0; r < NK; ++r) {
+      const int e = lane + 32 * r;
+      if (e < top_k - 1) ko[e] = e < keep ? m0[r] : 0ull;
+    }
+    pdl_release();
+    return;
+  }
   // element e = lane + 32 r holds rank e; sort the first `keep` by block index
   int blk[NK];
   float sc[NK];
@@ -976,7 +998,7 @@ static int pass1_slots(const void* fn, size_t smem) {
 
 template <typename T, int D, int KPL, int NST>
 static cudaError_t launch_pass1(const msa_paged_kv_t* kv, const void* q, int kw, int nch,
-                                uint64_t* lists, cudaStream_t st) {
+                                uint64_t* lists, int cand_lo, int cand_hi, cudaStream_t st) {
   const size_t smem = pass1_smem(kv, NST);
   auto k1 = select_decode_pass1<T, D, KPL, NST>;
   cudaError_t e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -988,62 +1010,92 @@ static cudaError_t launch_pass1(const msa_paged_kv_t* kv, const void* q, int kw,
                     (const float*)kv->centroids, (const int32_t*)kv->page_table,
                     (const int32_t*)kv->seq_lens, kv->status_word, kv->batch, kv->num_q_heads,
                     kv->num_kv_heads, hg, kv->block_size, kv->num_pages, kv->max_blocks_per_seq, kw,
-                    nch, lists);
+                    nch, cand_lo, cand_hi, lists);
 }
 
 template <typename T, int D, int NST>
 static cudaError_t pass1_dispatch_k(const msa_paged_kv_t* kv, const void* q, int kw, int nch,
-                                    uint64_t* lists, cudaStream_t st) {
+                                    uint64_t* lists, int lo, int hi, cudaStream_t st) {
   switch (kDecChunk / pass1_sc(pass1_groups(kv))) {
-    case 2: return launch_pass1<T, D, 2, NST>(kv, q, kw, nch, lists, st);
-    case 4: return launch_pass1<T, D, 4, NST>(kv, q, kw, nch, lists, st);
-    case 8: return launch_pass1<T, D, 8, NST>(kv, q, kw, nch, lists, st);
-    case 16: return launch_pass1<T, D, 16, 2>(kv, q, kw, nch, lists, st);
-    default: return launch_pass1<T, D, 32, 2>(kv, q, kw, nch, lists, st);
+    case 2: return launch_pass1<T, D, 2, NST>(kv, q, kw, nch, lists, lo, hi, st);
+    case 4: return launch_pass1<T, D, 4, NST>(kv, q, kw, nch, lists, lo, hi, st);
+    case 8: return launch_pass1<T, D, 8, NST>(kv, q, kw, nch, lists, lo, hi, st);
+    case 16: return launch_pass1<T, D, 16, 2>(kv, q, kw, nch, lists, lo, hi, st);
+    default: return launch_pass1<T, D, 32, 2>(kv, q, kw, nch, lists, lo, hi, st);
   }
+}
+
+// Merge launch: kw <= 32 and <= 64 keys per list use the merge tree; longer
+// lists (only for the per-sequence chunk lists) use the tournament.
+static cudaError_t launch_merge(const msa_paged_kv_t* kv, const uint64_t* lists, int kw, int nch,
+                                int top_k, int nlists, int lo, int hi, int32_t* idx, float* score,
+                                uint64_t* keys_out, cudaStream_t st) {
+  dim3 g2(kv->num_kv_heads, kv->batch);
+  const int32_t* sl = kv->seq_lens;
+  const int hkv = kv->num_kv_heads, B = kv->block_size, mb = kv->max_blocks_per_seq;
+  const int nl = nlists > 0 ? nlists : nch;
+  // lists per warp and round: enough that the four warps take them in one round
+  const int lg = nl <= 32 ? 8 : (nl <= 64 ? 16 : 32);
+  if (kw <= 32) {
+    auto k = lg == 8 ? select_decode_merge<1, 8>
+                     : (lg == 16 ? select_decode_merge<1, 16> : select_decode_merge<1, 32>);
+    return launch_pdl(k, g2, dim3(128), 0, st, lists, sl, kv->batch, hkv, B, mb, kw, nch, top_k,
+                      nlists, lo, hi, idx, score, keys_out);
+  }
+  auto k = lg == 8 ? select_decode_merge<2, 8> : select_decode_merge<2, 16>;
+  return launch_pdl(k, g2, dim3(128), 0, st, lists, sl, kv->batch, hkv, B, mb, kw, nch, top_k,
+                    nlists, lo, hi, idx, score, keys_out);
 }
 
 template <typename T, int D>
 static cudaError_t launch_decode_sel(const msa_paged_kv_t* kv, const void* q, int top_k,
-                                     int32_t* idx, float* score, void* ws, cudaStream_t st) {
+                                     int32_t* idx, float* score, void* ws, int lo, int hi,
+                                     uint64_t* keys_out, cudaStream_t st) {
   const int nch = decode_nchunks(kv), kw = decode_kw(top_k);
   uint64_t* lists = (uint64_t*)ws;
-  cudaError_t e = pass1_stages(kv) == 3 ? pass1_dispatch_k<T, D, 3>(kv, q, kw, nch, lists, st)
-                                        : pass1_dispatch_k<T, D, 2>(kv, q, kw, nch, lists, st);
+  cudaError_t e = pass1_stages(kv) == 3
+                      ? pass1_dispatch_k<T, D, 3>(kv, q, kw, nch, lists, lo, hi, st)
+                      : pass1_dispatch_k<T, D, 2>(kv, q, kw, nch, lists, lo, hi, st);
   if (e != cudaSuccess) return e;
-  dim3 g2(kv->num_kv_heads, kv->batch);
-  const int32_t* sl = kv->seq_lens;
-  const int hkv = kv->num_kv_heads, B = kv->block_size, mb = kv->max_blocks_per_seq;
-  // lists per warp and round: enough that the four warps take them in one round
-  const int lg = nch <= 32 ? 8 : (nch <= 64 ? 16 : 32);
-  if (kw <= 32) {
-    auto k = lg == 8 ? select_decode_merge<1, 8>
-                     : (lg == 16 ? select_decode_merge<1, 16> : select_decode_merge<1, 32>);
-    return launch_pdl(k, g2, dim3(128), 0, st, (const uint64_t*)lists, sl, hkv, B, mb, kw, nch,
-                      top_k, idx, score);
-  }
-  if (top_k - 1 <= 64) {
-    auto k = lg == 8 ? select_decode_merge<2, 8> : select_decode_merge<2, 16>;
-    return launch_pdl(k, g2, dim3(128), 0, st, (const uint64_t*)lists, sl, hkv, B, mb, kw, nch,
-                      top_k, idx, score);
-  }
+  if (top_k - 1 <= 64)
+    return launch_merge(kv, lists, kw, nch, top_k, 0, lo, hi, idx, score, keys_out, st);
   const size_t smem2 = (size_t)nch * kw * 8;
   e = cudaFuncSetAttribute(select_decode_pass2, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem2);
   if (e != cudaSuccess) return e;
+  dim3 g2(kv->num_kv_heads, kv->batch);
   return launch_pdl(select_decode_pass2, g2, dim3(32), smem2, st, (const uint64_t*)lists,
                     (const int32_t*)kv->seq_lens, kv->num_kv_heads, kv->block_size,
                     kv->max_blocks_per_seq, kw, nch, top_k, idx, score);
 }
 
-cudaError_t select_decode(const msa_paged_kv_t* kv, const void* q, int top_k, int32_t* idx,
-                          float* score, void* ws, cudaStream_t st) {
+static cudaError_t decode_sel_any(const msa_paged_kv_t* kv, const void* q, int top_k, int32_t* idx,
+                                  float* score, void* ws, int lo, int hi, uint64_t* keys_out,
+                                  cudaStream_t st) {
   const bool bf = kv->dtype == MSA_DTYPE_BF16;
   if (kv->head_dim == 128)
-    return bf ? launch_decode_sel<bf16, 128>(kv, q, top_k, idx, score, ws, st)
-              : launch_decode_sel<float, 128>(kv, q, top_k, idx, score, ws, st);
-  return bf ? launch_decode_sel<bf16, 64>(kv, q, top_k, idx, score, ws, st)
-            : launch_decode_sel<float, 64>(kv, q, top_k, idx, score, ws, st);
+    return bf ? launch_decode_sel<bf16, 128>(kv, q, top_k, idx, score, ws, lo, hi, keys_out, st)
+              : launch_decode_sel<float, 128>(kv, q, top_k, idx, score, ws, lo, hi, keys_out, st);
+  return bf ? launch_decode_sel<bf16, 64>(kv, q, top_k, idx, score, ws, lo, hi, keys_out, st)
+            : launch_decode_sel<float, 64>(kv, q, top_k, idx, score, ws, lo, hi, keys_out, st);
+}
+
+cudaError_t select_decode(const msa_paged_kv_t* kv, const void* q, int top_k, int32_t* idx,
+                          float* score, void* ws, cudaStream_t st) {
+  return decode_sel_any(kv, q, top_k, idx, score, ws, 0, 0x7fffffff, nullptr, st);
+}
+
+// Context-sharded decode: this rank's best keys among candidates [lo, hi).
+cudaError_t select_decode_range(const msa_paged_kv_t* kv, const void* q, int top_k, int lo, int hi,
+                                uint64_t* keys_out, void* ws, cudaStream_t st) {
+  return decode_sel_any(kv, q, top_k, nullptr, nullptr, ws, lo, hi, keys_out, st);
+}
+
+// Context-sharded decode: the global selection from nlists gathered key lists.
+cudaError_t select_merge_lists(const msa_paged_kv_t* kv, const uint64_t* keys, int nlists,
+                               int top_k, int32_t* idx, float* score, cudaStream_t st) {
+  return launch_merge(kv, keys, top_k - 1, 0, top_k, nlists, 0, 0x7fffffff, idx, score, nullptr,
+                      st);
 }
 
 }  // namespace msa

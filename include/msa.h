@@ -328,6 +328,59 @@ msa_status_t msa_sparse_attn_decode_tokens(const msa_paged_kv_t* kv, const void*
                                            float softmax_scale, void* out, float* lse,
                                            msa_stream_t stream);
 
+/*
+ * Context-sharded decode: the blocks of every sequence are split over several
+ * ranks (GPUs) by block range, each rank holding the K/V pages and centroids
+ * of its range [block_lo, block_hi). "Sparse Attention for Long-Context LLMs:
+ * Evolution and Practical Deployment", section 8 (future directions) lists
+ * sharing index results across devices and layers; the split follows the
+ * method's own structure: a rank scores only its blocks, the ranks' best
+ * candidates are gathered and the global top-k picked from them, each rank
+ * attends over the chosen blocks it holds, and the partial results are merged
+ * by log-sum-exp. The gathers between ranks are the caller's (NCCL all-gather
+ * in the Python binding); these calls are the per-rank steps.
+ *
+ * A rank's cache: page_table[b][j] holds the page of GLOBAL block j when j is
+ * in the rank's range (other entries are not read), seq_lens the global
+ * lengths, the new token appended by the rank whose range holds it.
+ *
+ * msa_select_topk_range: decode rows (one per sequence, at seq_lens-1); the
+ *   candidates are the complete past blocks j in [block_lo, block_hi). Writes
+ *   cand_keys [batch][num_kv_heads][top_k-1] u64: the rank's best min(k-1,
+ *   candidates) selection keys, descending (0 pads). A key is the block's fp32
+ *   score in order-preserving bits << 32 | (0x7fffffff - j): one unsigned
+ *   compare orders (score desc, index asc). 1 <= top_k <= 65. Workspace as
+ *   for msa_select_topk with cu_q == NULL.
+ * msa_select_merge: cand_keys [num_lists][batch][num_kv_heads][top_k-1] (the
+ *   ranks' lists, gathered in rank order) -> block_idx / block_score exactly as
+ *   msa_select_topk would produce them for the unsharded sequence.
+ * msa_sparse_attn_decode_range: the decode attention restricted to the
+ *   selected blocks in [block_lo, block_hi): o_part [batch][num_q_heads]
+ *   [head_dim] fp32 (normalised over this rank's keys, 0 if none) and lse_part
+ *   [batch][num_q_heads] (natural log, -inf if none). Workspace as for
+ *   msa_sparse_attn_decode; bf16 and head_dim 128 only.
+ * msa_lse_merge: o_parts [num_parts][rows][head_dim] fp32 and lse_parts
+ *   [num_parts][rows] -> out [rows][head_dim] (out_dtype, RNE) and lse [rows]
+ *   (may be NULL): sum_p exp(lse_p - M) o_p / sum_p exp(lse_p - M).
+ */
+msa_status_t msa_select_topk_range(const msa_paged_kv_t* kv, const void* q, int32_t block_lo,
+                                   int32_t block_hi, int32_t top_k, uint64_t* cand_keys,
+                                   void* workspace, size_t workspace_bytes, msa_stream_t stream);
+
+msa_status_t msa_select_merge(const msa_paged_kv_t* kv, const uint64_t* cand_keys,
+                              int32_t num_lists, int32_t top_k, int32_t* block_idx,
+                              float* block_score, msa_stream_t stream);
+
+msa_status_t msa_sparse_attn_decode_range(const msa_paged_kv_t* kv, const void* q,
+                                          const int32_t* block_idx, int32_t top_k,
+                                          int32_t block_lo, int32_t block_hi, float softmax_scale,
+                                          float* o_part, float* lse_part, void* workspace,
+                                          size_t workspace_bytes, msa_stream_t stream);
+
+msa_status_t msa_lse_merge(const float* o_parts, const float* lse_parts, int32_t num_parts,
+                           int32_t rows, int32_t head_dim, int32_t out_dtype, void* out,
+                           float* lse, msa_stream_t stream);
+
 /* Scratch bytes that `op` needs for these sizes (num_rows / max_rows_per_seq
  * as passed to the op; batch and 1 for decode). 0 means no scratch. */
 size_t msa_workspace_size(msa_op_t op, const msa_paged_kv_t* kv, int32_t num_rows,
