@@ -37,7 +37,7 @@ EXPORTS = ("msa_build_block_cache", "msa_select_topk", "msa_sparse_attn_prefill"
            "msa_sparse_attn_decode_gated", "msa_sparse_attn_decode_noalloc", "msa_workspace_size",
            "msa_status_string", "msa_version", "msa_select_tokens", "msa_sparse_attn_decode_tokens",
            "msa_select_topk_range", "msa_select_merge", "msa_sparse_attn_decode_range",
-           "msa_lse_merge")
+           "msa_lse_merge", "msa_select_tokens_rows", "msa_sparse_attn_prefill_tokens")
 
 
 class MsaError(RuntimeError):
@@ -96,6 +96,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.msa_sparse_attn_decode_range.argtypes = [KV, P, P, I32, I32, I32, ctypes.c_float, P, P, P,
                                                  SZ, P]
     lib.msa_lse_merge.argtypes = [P, P, I32, I32, I32, I32, P, P, P]
+    lib.msa_select_tokens_rows.argtypes = [KV, P, P, P, I32, I32, I32, P, P, SZ, P]
+    lib.msa_sparse_attn_prefill_tokens.argtypes = [KV, P, P, I32, P, I32, ctypes.c_float, P, P, P]
     lib.msa_workspace_size.argtypes = [ctypes.c_int, KV, I32, I32, I32]
     lib.msa_workspace_size.restype = SZ
     lib.msa_status_string.argtypes = [ctypes.c_int]
@@ -105,7 +107,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                  "msa_sparse_attn_decode", "msa_sparse_attn_prefill_gated",
                  "msa_sparse_attn_decode_gated", "msa_sparse_attn_decode_noalloc",
                  "msa_select_tokens", "msa_sparse_attn_decode_tokens", "msa_select_topk_range",
-                 "msa_select_merge", "msa_sparse_attn_decode_range", "msa_lse_merge"):
+                 "msa_select_merge", "msa_sparse_attn_decode_range", "msa_lse_merge",
+                 "msa_select_tokens_rows", "msa_sparse_attn_prefill_tokens"):
         getattr(lib, name).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -365,6 +368,47 @@ def select_tokens(cache: PagedKVCache, ki_pages: torch.Tensor, qi: torch.Tensor,
                                  _ptr(tok_idx), _ptr(ws), ws_bytes, _stream(stream)),
            "msa_select_tokens")
     return tok_idx
+
+
+def select_tokens_rows(cache: PagedKVCache, ki_pages: torch.Tensor, qi: torch.Tensor, top_k: int,
+                       cu_q: torch.Tensor, max_rows_per_seq: int,
+                       tok_idx: Optional[torch.Tensor] = None,
+                       workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Token-granular selection for many rows per sequence (prefill): qi
+    [rows, num_index_heads, head_dim]; the rows of sequence b are its last n_b
+    positions (cu_q as for select_topk). Returns tok_idx [rows, top_k]."""
+    lib = load_library()
+    _require_cuda(ki_pages, qi, cu_q, tok_idx)
+    rows = qi.shape[0]
+    if tok_idx is None:
+        tok_idx = torch.empty(rows, top_k, dtype=torch.int32, device=qi.device)
+    ws, ws_bytes = _workspace(MSA_OP_SELECT_TOKENS, cache, rows, max(2, max_rows_per_seq), top_k,
+                              workspace)
+    kv = cache.struct()
+    _check(lib.msa_select_tokens_rows(ctypes.byref(kv), _ptr(ki_pages), _ptr(qi), _ptr(cu_q), rows,
+                                      qi.shape[1], top_k, _ptr(tok_idx), _ptr(ws), ws_bytes,
+                                      _stream(stream)), "msa_select_tokens_rows")
+    return tok_idx
+
+
+def sparse_attn_prefill_tokens(cache: PagedKVCache, q: torch.Tensor, tok_idx: torch.Tensor,
+                               cu_q: torch.Tensor, softmax_scale: Optional[float] = None,
+                               out: Optional[torch.Tensor] = None,
+                               lse: Optional[torch.Tensor] = None, stream=None):
+    """Attention of each prefill row over its own kept positions."""
+    lib = load_library()
+    _require_cuda(q, tok_idx, cu_q, out, lse)
+    top_k = tok_idx.shape[-1]
+    scale = 1.0 / math.sqrt(cache.head_dim) if softmax_scale is None else softmax_scale
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(q.shape[0], q.shape[1], dtype=torch.float32, device=q.device)
+    kv = cache.struct()
+    _check(lib.msa_sparse_attn_prefill_tokens(ctypes.byref(kv), _ptr(q), _ptr(cu_q), q.shape[0],
+                                              _ptr(tok_idx), top_k, scale, _ptr(out), _ptr(lse),
+                                              _stream(stream)), "msa_sparse_attn_prefill_tokens")
+    return out, lse
 
 
 def sparse_attn_decode_tokens(cache: PagedKVCache, q: torch.Tensor, tok_idx: torch.Tensor,

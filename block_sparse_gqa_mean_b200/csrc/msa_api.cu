@@ -23,11 +23,11 @@ cudaError_t attn_simt(const msa_paged_kv_t*, const void*, const int32_t*, int, c
 size_t decode_ws(const msa_paged_kv_t*, int top_k, int num_sms);
 cudaError_t decode_splitk(const msa_paged_kv_t*, const void*, const int32_t*, int, float, void*,
                           float*, void*, int, gate_t, cudaStream_t);
-size_t tokens_ws(const msa_paged_kv_t*);
+size_t tokens_ws(const msa_paged_kv_t*, int num_rows);
 cudaError_t select_tokens(const msa_paged_kv_t*, const void*, const void*, int, int, int32_t*, void*,
-                          cudaStream_t);
+                          const int32_t*, int, cudaStream_t);
 cudaError_t attn_tokens(const msa_paged_kv_t*, const void*, const int32_t*, int, float, void*,
-                        float*, cudaStream_t);
+                        float*, const int32_t*, int, cudaStream_t);
 cudaError_t select_decode_range(const msa_paged_kv_t*, const void*, int, int, int, uint64_t*, void*,
                                 cudaStream_t);
 cudaError_t select_merge_lists(const msa_paged_kv_t*, const uint64_t*, int, int, int32_t*, float*,
@@ -146,9 +146,9 @@ const char* msa_status_string(msa_status_t s) {
 
 size_t msa_workspace_size(msa_op_t op, const msa_paged_kv_t* kv, int32_t num_rows,
                           int32_t max_rows_per_seq, int32_t top_k) {
-  (void)num_rows;
   if (check_kv(kv) != MSA_OK || top_k < 1) return 0;
-  if (op == MSA_OP_SELECT_TOKENS) return tokens_ws(kv);  // token top-K is not bounded by 256
+  if (op == MSA_OP_SELECT_TOKENS)  // token top-K is not bounded by 256
+    return tokens_ws(kv, max_rows_per_seq <= 1 ? kv->batch : (num_rows > 0 ? num_rows : 0));
   if (top_k > 256) return 0;
   switch (op) {
     case MSA_OP_SELECT:
@@ -305,34 +305,76 @@ msa_status_t msa_sparse_attn_decode_gated(const msa_paged_kv_t* kv, const void* 
 // ---------------------------------------------------------------------------
 extern "C" {
 
+static msa_status_t select_tokens_any(const msa_paged_kv_t* kv, const void* ki_pages,
+                                      const void* qi, const int32_t* cu_q, int32_t num_rows,
+                                      int32_t num_index_heads, int32_t top_k, int32_t* tok_idx,
+                                      void* workspace, size_t workspace_bytes,
+                                      msa_stream_t stream) {
+  msa_status_t s = msa::check_kv(kv);
+  if (s != MSA_OK) return s;
+  if (top_k < 1 || num_index_heads < 1 || num_index_heads > 256 || num_rows < 0 ||
+      num_rows > 65535)
+    return MSA_ERR_INVALID_ARG;
+  if (num_rows == 0) return MSA_OK;
+  if (!ki_pages || !qi || !tok_idx || !msa::aligned(ki_pages, 16) || !msa::aligned(qi, 16) ||
+      !msa::aligned(tok_idx, 4) || (cu_q && !msa::aligned(cu_q, 4)))
+    return MSA_ERR_INVALID_ARG;
+  const size_t need = msa::tokens_ws(kv, num_rows);
+  if (workspace_bytes < need || !workspace || !msa::aligned(workspace, 16)) return MSA_ERR_WORKSPACE;
+  return msa::from_cuda(msa::select_tokens(kv, ki_pages, qi, num_index_heads, top_k, tok_idx,
+                                           workspace, cu_q, num_rows, (cudaStream_t)stream));
+}
+
+static msa_status_t attn_tokens_any(const msa_paged_kv_t* kv, const void* q, const int32_t* cu_q,
+                                    int32_t num_rows, const int32_t* tok_idx, int32_t top_k,
+                                    float softmax_scale, void* out, float* lse,
+                                    msa_stream_t stream) {
+  msa_status_t s = msa::check_kv(kv);
+  if (s != MSA_OK) return s;
+  if (top_k < 1 || num_rows < 0 || num_rows > 65535) return MSA_ERR_INVALID_ARG;
+  if (num_rows == 0) return MSA_OK;
+  if (!q || !tok_idx || !out || !msa::aligned(q, 16) || !msa::aligned(out, 16) ||
+      !msa::aligned(tok_idx, 4) || (lse && !msa::aligned(lse, 4)) || (cu_q && !msa::aligned(cu_q, 4)) ||
+      !(softmax_scale > 0.f))
+    return MSA_ERR_INVALID_ARG;
+  return msa::from_cuda(msa::attn_tokens(kv, q, tok_idx, top_k, softmax_scale, out, lse, cu_q,
+                                         num_rows, (cudaStream_t)stream));
+}
+
 msa_status_t msa_select_tokens(const msa_paged_kv_t* kv, const void* ki_pages, const void* qi,
                                int32_t num_index_heads, int32_t top_k, int32_t* tok_idx,
                                void* workspace, size_t workspace_bytes, msa_stream_t stream) {
-  msa_status_t s = msa::check_kv(kv);
-  if (s != MSA_OK) return s;
-  if (top_k < 1 || num_index_heads < 1 || num_index_heads > 256) return MSA_ERR_INVALID_ARG;
-  if (!ki_pages || !qi || !tok_idx || !msa::aligned(ki_pages, 16) || !msa::aligned(qi, 16) ||
-      !msa::aligned(tok_idx, 4))
-    return MSA_ERR_INVALID_ARG;
-  const size_t need = msa::tokens_ws(kv);
-  if (workspace_bytes < need || !workspace || !msa::aligned(workspace, 16)) return MSA_ERR_WORKSPACE;
-  return msa::from_cuda(msa::select_tokens(kv, ki_pages, qi, num_index_heads, top_k, tok_idx,
-                                           workspace, (cudaStream_t)stream));
+  if (!kv) return MSA_ERR_INVALID_ARG;
+  return select_tokens_any(kv, ki_pages, qi, nullptr, kv->batch, num_index_heads, top_k, tok_idx,
+                           workspace, workspace_bytes, stream);
 }
 
 msa_status_t msa_sparse_attn_decode_tokens(const msa_paged_kv_t* kv, const void* q,
                                            const int32_t* tok_idx, int32_t top_k,
                                            float softmax_scale, void* out, float* lse,
                                            msa_stream_t stream) {
-  msa_status_t s = msa::check_kv(kv);
-  if (s != MSA_OK) return s;
-  if (top_k < 1) return MSA_ERR_INVALID_ARG;
-  if (kv->num_q_heads / kv->num_kv_heads > 16) return MSA_ERR_UNSUPPORTED;
-  if (!q || !tok_idx || !out || !msa::aligned(q, 16) || !msa::aligned(out, 16) ||
-      !msa::aligned(tok_idx, 4) || (lse && !msa::aligned(lse, 4)) || !(softmax_scale > 0.f))
-    return MSA_ERR_INVALID_ARG;
-  return msa::from_cuda(msa::attn_tokens(kv, q, tok_idx, top_k, softmax_scale, out, lse,
-                                         (cudaStream_t)stream));
+  if (!kv) return MSA_ERR_INVALID_ARG;
+  return attn_tokens_any(kv, q, nullptr, kv->batch, tok_idx, top_k, softmax_scale, out, lse,
+                         stream);
+}
+
+msa_status_t msa_select_tokens_rows(const msa_paged_kv_t* kv, const void* ki_pages,
+                                    const void* qi, const int32_t* cu_q, int32_t num_rows,
+                                    int32_t num_index_heads, int32_t top_k, int32_t* tok_idx,
+                                    void* workspace, size_t workspace_bytes,
+                                    msa_stream_t stream) {
+  if (!cu_q) return MSA_ERR_INVALID_ARG;
+  return select_tokens_any(kv, ki_pages, qi, cu_q, num_rows, num_index_heads, top_k, tok_idx,
+                           workspace, workspace_bytes, stream);
+}
+
+msa_status_t msa_sparse_attn_prefill_tokens(const msa_paged_kv_t* kv, const void* q,
+                                            const int32_t* cu_q, int32_t num_rows,
+                                            const int32_t* tok_idx, int32_t top_k,
+                                            float softmax_scale, void* out, float* lse,
+                                            msa_stream_t stream) {
+  if (!cu_q) return MSA_ERR_INVALID_ARG;
+  return attn_tokens_any(kv, q, cu_q, num_rows, tok_idx, top_k, softmax_scale, out, lse, stream);
 }
 
 }  // extern "C"

@@ -72,6 +72,30 @@ __device__ __forceinline__ unsigned block_scan_1024(unsigned v, unsigned* warp_t
   return r;
 }
 
+// Row r of a token-variant call: its sequence b and position t. Without cu_q
+// there is one row per sequence, at seq_lens[r] - 1 (decode); with cu_q the
+// rows cu_q[b] .. cu_q[b+1]-1 of sequence b sit at its last n_b positions
+// (prefill, chunked prefill). false: the sequence's length is not valid.
+__device__ __forceinline__ bool token_row(int r, const int32_t* __restrict__ cu_q, int batch,
+                                          const int32_t* __restrict__ seq_lens, int max_blocks,
+                                          int B, int& b, int& t) {
+  if (!cu_q) {
+    b = r;
+    t = seq_lens[r] - 1;
+    return t >= 0 && t < max_blocks * B;
+  }
+  int lo = 0, hi = batch;  // cu_q[lo] <= r < cu_q[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (cu_q[mid] <= r) lo = mid; else hi = mid;
+  }
+  b = lo;
+  const int n_b = cu_q[lo + 1] - cu_q[lo];
+  const int L = seq_lens[lo];
+  t = L - n_b + (r - cu_q[lo]);
+  return n_b <= L && L <= max_blocks * B && t >= 0;
+}
+
 }  // namespace
 
 // Scores of the earlier positions. A warp takes 32 consecutive positions; in
@@ -84,24 +108,24 @@ __device__ __forceinline__ unsigned block_scan_1024(unsigned v, unsigned* warp_t
 template <typename T, int D>
 __global__ void __launch_bounds__(256) tok_score_kernel(
     const T* __restrict__ qi, const T* __restrict__ ki_pages, const int32_t* __restrict__ page_table,
-    const int32_t* __restrict__ seq_lens, uint32_t* status, int hi, int B, int num_pages,
-    int max_blocks, int max_len, float* __restrict__ scores) {
+    const int32_t* __restrict__ seq_lens, const int32_t* __restrict__ cu_q, int batch,
+    uint32_t* status, int hi, int B, int num_pages, int max_blocks, int max_len,
+    float* __restrict__ scores) {
   constexpr int VEC = 16 / sizeof(T);       // elements per 16-byte chunk
   constexpr int CPR = D / VEC;              // chunks per row (16 for bf16 d 128)
   constexpr int RPI = 32 / CPR;             // rows per warp step
   static_assert(32 % CPR == 0, "a row's chunks stay inside one warp");
   __shared__ __align__(16) float qbar_s[D];
-  const int b = blockIdx.y;
-  const int L = seq_lens[b];
-  if (L < 1 || L > max_blocks * B) {
+  const int r = blockIdx.y;  // the query row
+  int b, t;                  // its sequence and position: positions 0 .. t-1 are scored
+  if (!token_row(r, cu_q, batch, seq_lens, max_blocks, B, b, t)) {
     if (blockIdx.x == 0 && threadIdx.x == 0) report(status, MSA_DEV_BAD_LENGTH);
     return;
   }
-  const int t = L - 1;  // the query's position: positions 0 .. t-1 are scored
   const int u_cta = blockIdx.x * kScoreChunk;
   if (u_cta >= t) return;
   for (int i = threadIdx.x; i < D; i += blockDim.x) {
-    const T* p = qi + (size_t)b * hi * D + i;
+    const T* p = qi + (size_t)r * hi * D + i;
     float s = to_f32(p[0]);
     for (int h = 1; h < hi; ++h) s = __fadd_rn(s, to_f32(p[(size_t)h * D]));
     qbar_s[i] = s;
@@ -143,31 +167,32 @@ __global__ void __launch_bounds__(256) tok_score_kernel(
         if (lane == step * RPI + r) res = v;
       }
     }
-    if (u0 + lane < t) scores[(size_t)b * max_len + u0 + lane] = res;
+    if (u0 + lane < t) scores[(size_t)r * max_len + u0 + lane] = res;
   }
 }
 
 __global__ void __launch_bounds__(kSelThreads) tok_select_kernel(
-    const float* __restrict__ scores, const int32_t* __restrict__ seq_lens, int max_blocks, int B,
-    int max_len, int top_k, int32_t* __restrict__ tok_idx) {
+    const float* __restrict__ scores, const int32_t* __restrict__ seq_lens,
+    const int32_t* __restrict__ cu_q, int batch, int max_blocks, int B, int max_len, int top_k,
+    int32_t* __restrict__ tok_idx) {
   __shared__ unsigned hist[256];
   __shared__ unsigned whist[256 * kSelWarps];  // per-warp histograms
   __shared__ unsigned warp_tot[33];
   __shared__ unsigned s_prefix, s_remaining;
-  const int b = blockIdx.x, tid = threadIdx.x;
-  const int L = seq_lens[b];
-  int32_t* out = tok_idx + (size_t)b * top_k;
-  if (L < 1 || L > max_blocks * B) {  // reported by the score kernel
+  const int r = blockIdx.x, tid = threadIdx.x;
+  int32_t* out = tok_idx + (size_t)r * top_k;
+  int b, t;
+  if (!token_row(r, cu_q, batch, seq_lens, max_blocks, B, b, t)) {  // reported by the score kernel
     for (int i = tid; i < top_k; i += kSelThreads) out[i] = -1;
     return;
   }
-  const int t = L - 1, n = t;  // candidates: the earlier positions 0 .. t-1
+  const int n = t;  // candidates: the earlier positions 0 .. t-1
   const int keep = min(top_k - 1, n);
   if (keep == n) {
     for (int i = tid; i < top_k; i += kSelThreads) out[i] = i < n ? i : (i == n ? t : -1);
     return;
   }
-  const float* sc = scores + (size_t)b * max_len;
+  const float* sc = scores + (size_t)r * max_len;
   // radix select: the key of the keep-th largest score, and how many keys equal
   // to it are kept (the lowest positions among them)
   unsigned prefix = 0u, pmask = 0u, remaining = (unsigned)keep;
@@ -251,7 +276,8 @@ __global__ void __launch_bounds__(kSelThreads) tok_select_kernel(
 template <typename T, int D>
 __global__ void __launch_bounds__(128) tok_attn_kernel(
     const T* __restrict__ q, const T* __restrict__ k_pages, const T* __restrict__ v_pages,
-    const int32_t* __restrict__ page_table, const int32_t* __restrict__ seq_lens, uint32_t* status,
+    const int32_t* __restrict__ page_table, const int32_t* __restrict__ seq_lens,
+    const int32_t* __restrict__ cu_q, int batch, uint32_t* status,
     const int32_t* __restrict__ tok_idx, int top_k, int hq, int hkv, int B, int num_pages,
     int max_blocks, float scale, T* __restrict__ out, float* __restrict__ lse) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -264,23 +290,22 @@ __global__ void __launch_bounds__(128) tok_attn_kernel(
   __shared__ float m_s[16], l_s[16], a_s[16];
   __shared__ int s_row[kTokChunk];                 // K/V row offset of each gathered token, -1: none
 
-  const int g = blockIdx.x, b = blockIdx.y;
+  const int g = blockIdx.x, r = blockIdx.y;
   const int tid = threadIdx.x;
-  const int L = seq_lens[b];
-  if (L < 1 || L > max_blocks * B) {
+  int b, t;
+  if (!token_row(r, cu_q, batch, seq_lens, max_blocks, B, b, t)) {
     if (tid == 0) report(status, MSA_DEV_BAD_LENGTH);
     return;
   }
-  const int t = L - 1;
   for (int e = tid; e < G * D; e += blockDim.x) {
-    qs[e] = to_f32(q[((size_t)b * hq + g * G) * D + e]);
+    qs[e] = to_f32(q[((size_t)r * hq + g * G) * D + e]);
     os[e] = 0.f;
   }
   if (tid < G) {
     m_s[tid] = -INFINITY;
     l_s[tid] = 0.f;
   }
-  const int32_t* list = tok_idx + (size_t)b * top_k;
+  const int32_t* list = tok_idx + (size_t)r * top_k;
   for (int c0 = 0; c0 < top_k; c0 += kTokChunk) {
     __syncthreads();  // the previous chunk fully consumed
     if (tid < kTokChunk) {
@@ -350,10 +375,10 @@ __global__ void __launch_bounds__(128) tok_attn_kernel(
   __syncthreads();
   for (int e = tid; e < G * D; e += blockDim.x) {
     const int h = e / D;
-    out[((size_t)b * hq + g * G) * D + e] = from_f32<T>(l_s[h] > 0.f ? os[e] / l_s[h] : 0.f);
+    out[((size_t)r * hq + g * G) * D + e] = from_f32<T>(l_s[h] > 0.f ? os[e] / l_s[h] : 0.f);
   }
   if (lse && tid < G)
-    lse[(size_t)b * hq + g * G + tid] = l_s[tid] > 0.f ? m_s[tid] + logf(l_s[tid]) : -INFINITY;
+    lse[(size_t)r * hq + g * G + tid] = l_s[tid] > 0.f ? m_s[tid] + logf(l_s[tid]) : -INFINITY;
 }
 
 constexpr int kTokTile = 64;    // tokens per stage of the tensor-core attention
@@ -379,7 +404,8 @@ __device__ __forceinline__ void cp_async_wait() {
 // zero-filled and masked. Warp w scores keys [16 w, 16 w + 16) of each stage.
 __global__ void __launch_bounds__(128) tok_attn_tc_kernel(
     const bf16* __restrict__ q, const bf16* __restrict__ k_pages, const bf16* __restrict__ v_pages,
-    const int32_t* __restrict__ page_table, const int32_t* __restrict__ seq_lens, uint32_t* status,
+    const int32_t* __restrict__ page_table, const int32_t* __restrict__ seq_lens,
+    const int32_t* __restrict__ cu_q, int batch, uint32_t* status,
     const int32_t* __restrict__ tok_idx, int top_k, int hq, int hkv, int B, int num_pages,
     int max_blocks, float scale_log2, bf16* __restrict__ out, float* __restrict__ lse) {
   using namespace warpmma;
@@ -391,14 +417,13 @@ __global__ void __launch_bounds__(128) tok_attn_tc_kernel(
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   __shared__ int s_row[kTokStages][kTokTile];  // K/V row of each slot, -1: none
-  const int g = blockIdx.x, b = blockIdx.y;
+  const int g = blockIdx.x, r = blockIdx.y;
   const int G = hq / hkv;
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-  const int L = seq_lens[b];
-  const bool len_ok = L >= 1 && L <= max_blocks * B;
+  int b, t;
+  const bool len_ok = token_row(r, cu_q, batch, seq_lens, max_blocks, B, b, t);
   if (!len_ok && g == 0 && tid == 0) report(status, MSA_DEV_BAD_LENGTH);
-  const int t = L - 1;
-  const int32_t* list = tok_idx + (size_t)b * top_k;
+  const int32_t* list = tok_idx + (size_t)r * top_k;
   const int nstage = len_ok ? (top_k + kTokTile - 1) / kTokTile : 0;
 
   // slot lookup for stage i (thread tid < 64: slot tid), then 16-byte copies:
@@ -436,7 +461,7 @@ __global__ void __launch_bounds__(128) tok_attn_tc_kernel(
   uint32_t qa[8][4];
   {
     const int r0 = lane / 4, r1 = r0 + 8, c = 2 * (lane % 4);
-    const bf16* qb = q + ((size_t)b * hq + (size_t)g * G) * D;
+    const bf16* qb = q + ((size_t)r * hq + (size_t)g * G) * D;
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) {
       const int k0 = ks * 16 + c;
@@ -567,20 +592,20 @@ __global__ void __launch_bounds__(128) tok_attn_tc_kernel(
     red_o[(warp * 16 + r1) * D + c + 1] = o[nd][3];
   }
   __syncthreads();
-  for (int r = 0; r < G; ++r) {
+  for (int hh = 0; hh < G; ++hh) {
     float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < 4; ++w) M = fmaxf(M, red_m[w * 16 + r]);
+    for (int w = 0; w < 4; ++w) M = fmaxf(M, red_m[w * 16 + hh]);
     float acc = 0.f, lsum = 0.f;
     if (M != -INFINITY) {
 #pragma unroll
       for (int w = 0; w < 4; ++w) {
-        const float f = exp2f(red_m[w * 16 + r] - M);
-        acc += f * red_o[(w * 16 + r) * D + tid];
-        lsum += f * red_l[w * 16 + r];
+        const float f = exp2f(red_m[w * 16 + hh] - M);
+        acc += f * red_o[(w * 16 + hh) * D + tid];
+        lsum += f * red_l[w * 16 + hh];
       }
     }
-    const size_t head = (size_t)b * hq + (size_t)g * G + r;
+    const size_t head = (size_t)r * hq + (size_t)g * G + hh;
     out[head * D + tid] = __float2bfloat16_rn(lsum > 0.f ? acc / lsum : 0.f);
     if (lse && tid == 0) lse[head] = lsum > 0.f ? (M + log2f(lsum)) * 0.6931471805599453f : -INFINITY;
   }
@@ -589,58 +614,62 @@ __global__ void __launch_bounds__(128) tok_attn_tc_kernel(
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-size_t tokens_ws(const msa_paged_kv_t* kv) {
-  return (size_t)kv->batch * kv->max_blocks_per_seq * kv->block_size * sizeof(float);
+// one fp32 score per (row, position)
+size_t tokens_ws(const msa_paged_kv_t* kv, int num_rows) {
+  return (size_t)num_rows * kv->max_blocks_per_seq * kv->block_size * sizeof(float);
 }
 
 template <typename T, int D>
 static cudaError_t launch_tok_select(const msa_paged_kv_t* kv, const void* ki_pages, const void* qi,
                                      int hi, int top_k, int32_t* tok_idx, void* ws,
-                                     cudaStream_t st) {
+                                     const int32_t* cu_q, int rows, cudaStream_t st) {
   const int max_len = kv->max_blocks_per_seq * kv->block_size;
   float* scores = (float*)ws;
-  dim3 grid((max_len + kScoreChunk - 1) / kScoreChunk, kv->batch);
+  dim3 grid((max_len + kScoreChunk - 1) / kScoreChunk, rows);
   tok_score_kernel<T, D><<<grid, 256, 0, st>>>((const T*)qi, (const T*)ki_pages, kv->page_table,
-                                               kv->seq_lens, kv->status_word, hi, kv->block_size,
-                                               kv->num_pages, kv->max_blocks_per_seq, max_len,
-                                               scores);
+                                               kv->seq_lens, cu_q, kv->batch, kv->status_word, hi,
+                                               kv->block_size, kv->num_pages,
+                                               kv->max_blocks_per_seq, max_len, scores);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  tok_select_kernel<<<kv->batch, kSelThreads, 0, st>>>(scores, kv->seq_lens,
-                                                       kv->max_blocks_per_seq, kv->block_size,
-                                                       max_len, top_k, tok_idx);
+  tok_select_kernel<<<rows, kSelThreads, 0, st>>>(scores, kv->seq_lens, cu_q, kv->batch,
+                                                  kv->max_blocks_per_seq, kv->block_size, max_len,
+                                                  top_k, tok_idx);
   return cudaGetLastError();
 }
 
 cudaError_t select_tokens(const msa_paged_kv_t* kv, const void* ki_pages, const void* qi, int hi,
-                          int top_k, int32_t* tok_idx, void* ws, cudaStream_t st) {
+                          int top_k, int32_t* tok_idx, void* ws, const int32_t* cu_q, int rows,
+                          cudaStream_t st) {
   const bool bf = kv->dtype == MSA_DTYPE_BF16;
   if (kv->head_dim == 128)
-    return bf ? launch_tok_select<bf16, 128>(kv, ki_pages, qi, hi, top_k, tok_idx, ws, st)
-              : launch_tok_select<float, 128>(kv, ki_pages, qi, hi, top_k, tok_idx, ws, st);
-  return bf ? launch_tok_select<bf16, 64>(kv, ki_pages, qi, hi, top_k, tok_idx, ws, st)
-            : launch_tok_select<float, 64>(kv, ki_pages, qi, hi, top_k, tok_idx, ws, st);
+    return bf ? launch_tok_select<bf16, 128>(kv, ki_pages, qi, hi, top_k, tok_idx, ws, cu_q, rows, st)
+              : launch_tok_select<float, 128>(kv, ki_pages, qi, hi, top_k, tok_idx, ws, cu_q, rows, st);
+  return bf ? launch_tok_select<bf16, 64>(kv, ki_pages, qi, hi, top_k, tok_idx, ws, cu_q, rows, st)
+            : launch_tok_select<float, 64>(kv, ki_pages, qi, hi, top_k, tok_idx, ws, cu_q, rows, st);
 }
 
 template <typename T, int D>
 static cudaError_t launch_tok_attn(const msa_paged_kv_t* kv, const void* q, const int32_t* tok_idx,
-                                   int top_k, float scale, void* out, float* lse, cudaStream_t st) {
+                                   int top_k, float scale, void* out, float* lse,
+                                   const int32_t* cu_q, int rows, cudaStream_t st) {
   const int G = kv->num_q_heads / kv->num_kv_heads;
   const size_t smem = ((size_t)2 * G * D + (size_t)kTokChunk * (D + 1) + (size_t)kTokChunk * D +
                        (size_t)G * kTokChunk) * 4;
   auto kern = tok_attn_kernel<T, D>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  dim3 grid(kv->num_kv_heads, kv->batch);
+  dim3 grid(kv->num_kv_heads, rows);
   kern<<<grid, 128, smem, st>>>((const T*)q, (const T*)kv->k_pages, (const T*)kv->v_pages,
-                                 kv->page_table, kv->seq_lens, kv->status_word, tok_idx, top_k,
-                                 kv->num_q_heads, kv->num_kv_heads, kv->block_size, kv->num_pages,
-                                 kv->max_blocks_per_seq, scale, (T*)out, lse);
+                                 kv->page_table, kv->seq_lens, cu_q, kv->batch, kv->status_word,
+                                 tok_idx, top_k, kv->num_q_heads, kv->num_kv_heads, kv->block_size,
+                                 kv->num_pages, kv->max_blocks_per_seq, scale, (T*)out, lse);
   return cudaGetLastError();
 }
 
 cudaError_t attn_tokens(const msa_paged_kv_t* kv, const void* q, const int32_t* tok_idx, int top_k,
-                        float scale, void* out, float* lse, cudaStream_t st) {
+                        float scale, void* out, float* lse, const int32_t* cu_q, int rows,
+                        cudaStream_t st) {
   const bool bf = kv->dtype == MSA_DTYPE_BF16;
   if (bf && kv->head_dim == 128) {
     const size_t red = (size_t)4 * 16 * 128 * 4 + 2 * 4 * 16 * 4;
@@ -649,19 +678,19 @@ cudaError_t attn_tokens(const msa_paged_kv_t* kv, const void* q, const int32_t* 
     cudaError_t e = cudaFuncSetAttribute(tok_attn_tc_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    dim3 grid(kv->num_kv_heads, kv->batch);
+    dim3 grid(kv->num_kv_heads, rows);
     tok_attn_tc_kernel<<<grid, 128, smem, st>>>(
         (const bf16*)q, (const bf16*)kv->k_pages, (const bf16*)kv->v_pages, kv->page_table,
-        kv->seq_lens, kv->status_word, tok_idx, top_k, kv->num_q_heads, kv->num_kv_heads,
-        kv->block_size, kv->num_pages, kv->max_blocks_per_seq, scale * 1.4426950408889634f,
-        (bf16*)out, lse);
+        kv->seq_lens, cu_q, kv->batch, kv->status_word, tok_idx, top_k, kv->num_q_heads,
+        kv->num_kv_heads, kv->block_size, kv->num_pages, kv->max_blocks_per_seq,
+        scale * 1.4426950408889634f, (bf16*)out, lse);
     return cudaGetLastError();
   }
   if (kv->head_dim == 128)
-    return bf ? launch_tok_attn<bf16, 128>(kv, q, tok_idx, top_k, scale, out, lse, st)
-              : launch_tok_attn<float, 128>(kv, q, tok_idx, top_k, scale, out, lse, st);
-  return bf ? launch_tok_attn<bf16, 64>(kv, q, tok_idx, top_k, scale, out, lse, st)
-            : launch_tok_attn<float, 64>(kv, q, tok_idx, top_k, scale, out, lse, st);
+    return bf ? launch_tok_attn<bf16, 128>(kv, q, tok_idx, top_k, scale, out, lse, cu_q, rows, st)
+              : launch_tok_attn<float, 128>(kv, q, tok_idx, top_k, scale, out, lse, cu_q, rows, st);
+  return bf ? launch_tok_attn<bf16, 64>(kv, q, tok_idx, top_k, scale, out, lse, cu_q, rows, st)
+            : launch_tok_attn<float, 64>(kv, q, tok_idx, top_k, scale, out, lse, cu_q, rows, st);
 }
 
 }  // namespace msa

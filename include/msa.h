@@ -329,6 +329,33 @@ msa_status_t msa_sparse_attn_decode_tokens(const msa_paged_kv_t* kv, const void*
                                            msa_stream_t stream);
 
 /*
+ * msa_select_tokens_rows / msa_sparse_attn_prefill_tokens - the same two
+ * steps for many query rows per sequence (prefill, chunked prefill): the rows
+ * cu_q[b] .. cu_q[b+1]-1 of sequence b sit at its last n_b positions, as for
+ * msa_select_topk with cu_q. Row r at position t scores the positions u < t
+ * and keeps t plus the best top_k-1 of them; the attention of row r runs over
+ * its own kept positions (rows share no keys, so each row gathers its own).
+ *
+ *   qi        : device [num_rows][num_index_heads][head_dim], kv->dtype.
+ *   q, out    : device [num_rows][num_q_heads][head_dim]; lse [num_rows][num_q_heads].
+ *   tok_idx   : device [num_rows][top_k] int32, ascending (t last), -1 padded.
+ *   workspace : msa_workspace_size(MSA_OP_SELECT_TOKENS, kv, num_rows,
+ *               max_rows_per_seq > 1, top_k) bytes: one fp32 score per row
+ *               and position (num_rows * max_blocks_per_seq * block_size * 4).
+ *   num_rows <= 65535; cu_q must not be NULL. Errors as for the decode form.
+ */
+msa_status_t msa_select_tokens_rows(const msa_paged_kv_t* kv, const void* ki_pages,
+                                    const void* qi, const int32_t* cu_q, int32_t num_rows,
+                                    int32_t num_index_heads, int32_t top_k, int32_t* tok_idx,
+                                    void* workspace, size_t workspace_bytes, msa_stream_t stream);
+
+msa_status_t msa_sparse_attn_prefill_tokens(const msa_paged_kv_t* kv, const void* q,
+                                            const int32_t* cu_q, int32_t num_rows,
+                                            const int32_t* tok_idx, int32_t top_k,
+                                            float softmax_scale, void* out, float* lse,
+                                            msa_stream_t stream);
+
+/*
  * Context-sharded decode: the blocks of every sequence are split over several
  * ranks (GPUs) by block range, each rank holding the K/V pages and centroids
  * of its range [block_lo, block_hi). "Sparse Attention for Long-Context LLMs:

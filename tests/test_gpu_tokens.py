@@ -111,3 +111,76 @@ def test_token_decode_repeated_and_empty_lists():
     assert cache.device_status() == 0
     assert (o3[0].float() - o4[0].float()).abs().max().item() < 1e-6
     assert torch.all(o3[1] == 0) and torch.all(torch.isneginf(l3[1]))
+
+
+# ---------------------------------------------------------------------------
+# prefill form: every row scores its own earlier positions
+# ---------------------------------------------------------------------------
+def _prefill_case():
+    w = workloads.prefill_bf16(batch=2, ctx=(700, 1200), block=64, top_k=4, hq=16, hkv=2)
+    p = workloads.paging(w)
+    cache = new_cache(w, p)
+    first = [0, 900]                                   # sequence 1: a chunk after 900 cached
+    append(cache, w, [0, 0], first)
+    append(cache, w, first, list(w.ctx))
+    ki = _index_pages(w, p, list(w.ctx))
+    n = [w.ctx[b] - first[b] for b in range(2)]
+    cu = msa.cu_seqlens(n, DEV)
+    q = torch.cat([workloads.queries_prefill(w, b, first[b], w.ctx[b], DEV) for b in range(2)])
+    gen = torch.Generator().manual_seed(11)
+    qi = (torch.randn(sum(n), HI, w.d, generator=gen) * 0.5).to(torch.bfloat16).to(DEV)
+    return w, cache, ki, first, n, cu, q, qi
+
+
+@pytest.mark.parametrize("top_k", [1, 64, 300, 5000])
+def test_token_prefill_selection_and_attention(top_k):
+    w, cache, ki, first, n, cu, q, qi = _prefill_case()
+    idx = msa.select_tokens_rows(cache, ki, qi, top_k, cu, max(n))
+    torch.cuda.synchronize()
+    assert cache.device_status() == 0
+    gi = idx.cpu().numpy()
+    oidx_all, refs, protected = [], [], 0
+    r0 = 0
+    for b in range(2):
+        L = w.ctx[b]
+        pos = np.arange(first[b], L)
+        KI = workloads.indexer_keys(w, b, 0, L)
+        S = oracle.token_scores(qi[r0:r0 + n[b]].cpu(), KI, pos)
+        oidx, gap = oracle.token_select(S, pos, top_k)
+        for i in range(n[b]):
+            row, t = gi[r0 + i], pos[i]
+            kept = [int(u) for u in row if u >= 0]
+            assert kept == sorted(set(kept)) and kept[-1] == t
+            assert len(kept) == min(top_k, t + 1) and np.all(row[len(kept):] == -1)
+            if gap[i] >= GAP_MIN:
+                protected += 1
+                assert np.array_equal(row, oidx[i]), (b, i)
+            elif not np.array_equal(row, oidx[i]):
+                earlier = [u for u in kept if u != t]
+                cut = np.sort(S[i, :t])[::-1][len(earlier) - 1]
+                assert all(S[i, u] >= cut - 1e-3 for u in earlier)
+        K, V = workloads.keys(w, b, 0, L), workloads.values(w, b, 0, L)
+        O, _ = oracle.attend_tokens(q[r0:r0 + n[b]].cpu(), K, V, pos, oidx, w.softmax_scale)
+        oidx_all.append(oidx)
+        refs.append(O)
+        r0 += n[b]
+    assert protected >= 0.8 * sum(n), protected
+    oi = torch.from_numpy(np.concatenate(oidx_all)).to(DEV)
+    out, lse = msa.sparse_attn_prefill_tokens(cache, q, oi, cu)
+    torch.cuda.synchronize()
+    assert cache.device_status() == 0
+    compare(out, np.concatenate(refs), w.dtype)
+
+
+def test_token_prefill_row_equals_decode_row():
+    """The prefill form's last row and the decode form of the same query agree."""
+    w, cache, ki, first, n, cu, q, qi = _prefill_case()
+    idx = msa.select_tokens_rows(cache, ki, qi, 64, cu, max(n))
+    out, _ = msa.sparse_attn_prefill_tokens(cache, q, idx, cu)
+    last = [n[0] - 1, n[0] + n[1] - 1]                 # each sequence's last row
+    qd, qid = q[last].contiguous(), qi[last].contiguous()
+    idx_d = msa.select_tokens(cache, ki, qid, 64)
+    out_d, _ = msa.sparse_attn_decode_tokens(cache, qd, idx_d)
+    torch.cuda.synchronize()
+    assert torch.equal(idx_d, idx[last])
+    assert torch.equal(out_d.view(torch.int16), out[last].view(torch.int16))
