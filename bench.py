@@ -72,6 +72,21 @@ def profile_traffic(kernel: str, src: str):
     return profile_value(kernel, src, "dram_bytes_per_full_launch")
 
 
+def tensor_pipe(executed_tflops, clocks):
+    """Tensor-pipe utilisation of the prefill attention kernel, two ways: the ncu
+    counter recorded in its profile (same source hash only), and the executed
+    MMA rate of this run against the hardware rate the counter is measured
+    against (one M128 N128 K16 bf16 MMA per 64 cycles = 8192 flops/cycle/SM on
+    148 SMs at the sampled SM clock)."""
+    mhz = clocks.get("sm_mhz") or 1965.0
+    hw_tflops = 148 * 8192 * mhz * 1e6 / 1e12
+    return {"ncu_active_pct": profile_value("prefill_tc_kernel", "prefill_tc.cu",
+                                            "tensor_pipe_active_pct"),
+            "ncu_case": "T=16384 capture of the same kernel (profiles/)",
+            "hw_rate_tflops": hw_tflops,
+            "executed_pct_of_hw_rate": 100.0 * executed_tflops / hw_tflops}
+
+
 def profile_value(kernel: str, src: str, key: str):
     """A figure `key: value` recorded in profiles/<kernel>*.md, if the kernel
     source still hashes to the recorded value; else None."""
@@ -872,7 +887,9 @@ def main():
                          "kernel": "msa_sparse_attn_prefill (cluster + plan + prefill_tc_kernel)",
                          "algorithmic_flops_per_launch": flops,
                          "executed_mma_flops_per_launch": executed,
-                         "executed_tflops": executed / (attn_ms * 1e-3) / 1e12},
+                         "executed_tflops": executed / (attn_ms * 1e-3) / 1e12,
+                         "tensor_pipe": tensor_pipe(executed / (attn_ms * 1e-3) / 1e12,
+                                                    r["clocks"])},
             "kernels_ms": {"build_block_cache": r["kernel_ms"][0], "select_topk": r["kernel_ms"][1],
                            "sparse_attn_prefill": r["kernel_ms"][2]},
             "e2e": {"value": T * world / (max_over_ranks(r["e2e_ms"], world) * 1e-3),
