@@ -25,19 +25,25 @@ from typing import Optional, Tuple
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_PKG, "libmsa.so")
+# MSA_LIBRARY may name another build of the library, e.g. the bounds-checked
+# libmsa_debug.so (python -m block_sparse_gqa_mean_b200.build --debug-bounds).
+LIB_PATH = os.environ.get("MSA_LIBRARY") or os.path.join(_PKG, "libmsa.so")
+DEBUG_LIB_PATH = os.path.join(_PKG, "libmsa_debug.so")
 
 MSA_OK, MSA_ERR_INVALID_ARG, MSA_ERR_UNSUPPORTED, MSA_ERR_WORKSPACE, MSA_ERR_CUDA = range(5)
 MSA_DTYPE_BF16, MSA_DTYPE_F32 = 0, 1
 MSA_OP_SELECT, MSA_OP_PREFILL, MSA_OP_DECODE, MSA_OP_SELECT_TOKENS = 0, 1, 2, 3
 MSA_DEV_BAD_PAGE, MSA_DEV_BAD_LENGTH, MSA_DEV_BAD_INDEX, MSA_DEV_TIMEOUT = 1, 2, 4, 8
+MSA_DEV_BOUNDS = 0x10
+MSA_BUILD_DEBUG_BOUNDS = 1
 
 EXPORTS = ("msa_build_block_cache", "msa_select_topk", "msa_sparse_attn_prefill",
            "msa_sparse_attn_decode", "msa_sparse_attn_prefill_gated",
            "msa_sparse_attn_decode_gated", "msa_sparse_attn_decode_noalloc", "msa_workspace_size",
            "msa_status_string", "msa_version", "msa_select_tokens", "msa_sparse_attn_decode_tokens",
            "msa_select_topk_range", "msa_select_merge", "msa_sparse_attn_decode_range",
-           "msa_lse_merge", "msa_select_tokens_rows", "msa_sparse_attn_prefill_tokens")
+           "msa_lse_merge", "msa_select_tokens_rows", "msa_sparse_attn_prefill_tokens",
+           "msa_build_flags")
 
 
 class MsaError(RuntimeError):
@@ -103,6 +109,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.msa_status_string.argtypes = [ctypes.c_int]
     lib.msa_status_string.restype = ctypes.c_char_p
     lib.msa_version.restype = I32
+    lib.msa_build_flags.restype = I32
     for name in ("msa_build_block_cache", "msa_select_topk", "msa_sparse_attn_prefill",
                  "msa_sparse_attn_decode", "msa_sparse_attn_prefill_gated",
                  "msa_sparse_attn_decode_gated", "msa_sparse_attn_decode_noalloc",
@@ -116,6 +123,12 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
 
 def status_string(status: int) -> str:
     return load_library().msa_status_string(status).decode()
+
+
+def build_flags() -> int:
+    """MSA_BUILD_* bits of the loaded library (MSA_BUILD_DEBUG_BOUNDS for
+    the bounds-checked build)."""
+    return int(load_library().msa_build_flags())
 
 
 def _ptr(t: Optional[torch.Tensor]):

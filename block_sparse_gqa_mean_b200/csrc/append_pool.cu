@@ -36,6 +36,11 @@ __global__ void __launch_bounds__(128) append_pool_kernel(
     return;
   }
   const int t0 = L - n_new;           // first new position
+  // the new rows lie inside k_new / v_new, and the grid (sized from the
+  // caller's max_new) covers every block they touch
+  if (!MSA_RANGE_OK(row0, row0 + n_new, cu_new[gridDim.y], status) ||
+      !MSA_RANGE_OK(0, (t0 % B + n_new + B - 1) / B, gridDim.x, status))
+    return;
   const int j = t0 / B + lb;          // logical block
   if (j * B >= L) return;             // beyond the last touched block
   const int page = page_table[(size_t)b * max_blocks + j];
@@ -56,6 +61,7 @@ __global__ void __launch_bounds__(128) append_pool_kernel(
     const int u = u_lo + r;
     const size_t src = ((size_t)(row0 + (u - t0)) * hkv + g) * D + col;
     const size_t dst = page_off + (size_t)(u - j * B) * D + col;
+    if (!MSA_RANGE_OK(dst, dst + VEC, (size_t)num_pages * hkv * B * D, status)) continue;
     *reinterpret_cast<uint4*>(k_pages + dst) = *reinterpret_cast<const uint4*>(k_new + src);
     *reinterpret_cast<uint4*>(v_pages + dst) = *reinterpret_cast<const uint4*>(v_new + src);
   }
@@ -67,8 +73,9 @@ __global__ void __launch_bounds__(128) append_pool_kernel(
   T* tile = reinterpret_cast<T*>(smem_raw);  // [n][D]
   const int n = u_hi - j * B;
   for (int c = threadIdx.x; c < n * CPR; c += blockDim.x)
-    reinterpret_cast<uint4*>(tile)[c] =
-        reinterpret_cast<const uint4*>(k_pages + page_off)[c];
+    if (MSA_IN_BOUNDS(c, B * CPR, status))
+      reinterpret_cast<uint4*>(tile)[c] =
+          reinterpret_cast<const uint4*>(k_pages + page_off)[c];
   __syncthreads();
   for (int i = threadIdx.x; i < D; i += blockDim.x) {
     float s = 0.f;

@@ -37,6 +37,9 @@ __global__ void __launch_bounds__(128) attn_simt_kernel(
   const int L = seq_lens[b];
   if (cu_q) {
     const int r0 = cu_q[b], n = cu_q[b + 1] - r0;
+    // the sequence's rows lie inside q / out, and the grid covers all of them
+    if (blockIdx.x == 0) (void)MSA_RANGE_OK(n, n, gridDim.x, status);
+    if (!MSA_RANGE_OK(r0, r0 + n, cu_q[gridDim.y], status)) return;
     if ((int)blockIdx.x >= n) return;
     row = r0 + blockIdx.x;
     if (n > L || L > max_blocks * B) {
@@ -77,6 +80,8 @@ __global__ void __launch_bounds__(128) attn_simt_kernel(
     }
     const int nk = min(B, t + 1 - j * B);
     const size_t base = ((size_t)page * hkv + g) * B * D;
+    if (!MSA_RANGE_OK(base, base + (size_t)nk * D, (size_t)num_pages * hkv * B * D, status))
+      continue;
     __syncthreads();  // previous block's K/V/P fully consumed
     for (int e = tid; e < nk * D; e += blockDim.x) {
       const int kk = e / D, i = e % D;

@@ -56,6 +56,33 @@ __device__ __forceinline__ void report(uint32_t* status, uint32_t bits) {
   if (status) atomicOr(status, bits);
 }
 
+// Bounds-checked build. Compiled with -DMSA_DEBUG_BOUNDS (libmsa_debug.so),
+// every index a kernel derives from device data or from a launch-size
+// assumption goes through MSA_IN_BOUNDS / MSA_RANGE_OK before the access it
+// guards: a failed check records MSA_DEV_BOUNDS and the caller skips the
+// access (or substitutes a valid index where a pipeline must stay in step).
+// In the regular build both macros are the constant true and their
+// arguments are not evaluated, so the checks cost nothing there.
+#ifdef MSA_DEBUG_BOUNDS
+constexpr bool kDebugBounds = true;
+__device__ __forceinline__ bool debug_range_ok(long long lo, long long hi, long long n,
+                                               uint32_t* status) {
+  const bool ok = 0 <= lo && lo <= hi && hi <= n;
+  if (!ok) report(status, MSA_DEV_BOUNDS);
+  return ok;
+}
+// 0 <= i < n
+#define MSA_IN_BOUNDS(i, n, status) \
+  ::msa::debug_range_ok((long long)(i), (long long)(i) + 1, (long long)(n), (status))
+// 0 <= lo <= hi <= n: the half-open range [lo, hi) lies inside [0, n)
+#define MSA_RANGE_OK(lo, hi, n, status) \
+  ::msa::debug_range_ok((long long)(lo), (long long)(hi), (long long)(n), (status))
+#else
+constexpr bool kDebugBounds = false;
+#define MSA_IN_BOUNDS(i, n, status) true
+#define MSA_RANGE_OK(lo, hi, n, status) true
+#endif
+
 template <typename T>
 __device__ __forceinline__ float to_f32(T x);
 template <>

@@ -94,7 +94,7 @@ __global__ void __launch_bounds__(128) decode_splitk_kernel(
     __syncthreads();
     int pos = s_n + __popc(bal & ((1u << lane) - 1u));
     for (int w = 0; w < warp; ++w) pos += s_wcnt[w];
-    if (ok) {
+    if (ok && MSA_IN_BOUNDS(pos, 256, status)) {
       s_page[pos] = pg;
       s_blk[pos] = j;
     }

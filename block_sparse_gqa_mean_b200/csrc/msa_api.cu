@@ -133,6 +133,8 @@ extern "C" {
 
 int32_t msa_version(void) { return 1000; }
 
+int32_t msa_build_flags(void) { return kDebugBounds ? MSA_BUILD_DEBUG_BOUNDS : 0; }
+
 const char* msa_status_string(msa_status_t s) {
   switch (s) {
     case MSA_OK: return "ok";

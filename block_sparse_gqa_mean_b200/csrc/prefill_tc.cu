@@ -172,7 +172,11 @@ __global__ void __launch_bounds__(128) prefill_plan_kernel(
   const int row0 = cu_q[b];
   const int n_rows = cu_q[b + 1] - row0;
   const int r_lo = tt * TM;
-  if (r_lo >= n_rows) {
+  // the sequence's rows lie inside q / block_idx, and the tiles cover all of them
+  if (tt == 0 && g == 0 && tid == 0)
+    (void)MSA_RANGE_OK(n_rows, n_rows, units_per_seq * TM, status);
+  if (r_lo >= n_rows ||
+      !MSA_RANGE_OK(row0, row0 + n_rows, cu_q[gridDim.x / (hkv * units_per_seq)], status)) {
     if (tid == 0) counts[tile] = 0;
     return;
   }
@@ -201,6 +205,7 @@ __global__ void __launch_bounds__(128) prefill_plan_kernel(
     for (int it = tid; it < nr * top_k; it += 128) {
       const int i = it / top_k, s = it % top_k;
       const int o = pw[p0 + i];                     // the token's offset in its window
+      if (!MSA_IN_BOUNDS(o, nw, status)) continue;
       const int j = block_idx[((size_t)(row0 + w * kWin + o) * hkv + g) * top_k + s];
       if (j < 0) continue;
       const int own_i = (t_win + o) / B;
@@ -226,12 +231,15 @@ __global__ void __launch_bounds__(128) prefill_plan_kernel(
     int off = s_base + incl - cnt;
     for (int w = 0; w < warp; ++w) off += warp_tot[w];
     for (int a = a0; a < a1; ++a)
-      if (bm[a] != 0u) out[off++] = make_int2(w0 + a, (int)bm[a]);
+      if (bm[a] != 0u) {
+        if (MSA_IN_BOUNDS(off, ecap, status)) out[off] = make_int2(w0 + a, (int)bm[a]);
+        ++off;
+      }
     __syncthreads();
     if (tid == 0) s_base += warp_tot[0] + warp_tot[1] + warp_tot[2] + warp_tot[3];
     __syncthreads();
   }
-  if (tid == 0) counts[tile] = s_base;
+  if (tid == 0) counts[tile] = MSA_RANGE_OK(s_base, s_base, ecap, status) ? s_base : 0;
 }
 
 // ---------------------------------------------------------------------------
@@ -352,7 +360,8 @@ __global__ void __launch_bounds__(192, 1) prefill_tc_kernel(
   const int g = unit % hkv;
   const int pu = (unit / hkv) % units_per_seq;
   const int b = unit / (hkv * units_per_seq);
-  const int n_e = counts[unit];
+  int n_e = counts[unit];
+  if (!MSA_RANGE_OK(n_e, n_e, ecap, status)) n_e = 0;
   const int2* ent = entries + (size_t)unit * ecap;
   const int row0 = cu_q[b];
   const int n_rows = cu_q[b + 1] - row0;
@@ -365,13 +374,18 @@ __global__ void __launch_bounds__(192, 1) prefill_tc_kernel(
   const int L = seq_lens[b];
   const int t_win = L - n_rows + wdw * kWin;      // position of the window's first row
   const int row_win = row0 + wdw * kWin;          // global row of the window's first row
+  // window offset of the tile's token ti (the order table is the library's own)
+  auto tok_off = [&](int ti) {
+    const int o = pw[p0 + ti];
+    return MSA_IN_BOUNDS(o, nw, status) ? o : 0;
+  };
   if (n_e == 0) {
     // no token of the tile took a block (or the tile lies past the sequence's
     // rows): its rows attend to nothing, A = 0. Uniform exit before any sync.
     if (threadIdx.x >= 64) {
       const int r = threadIdx.x - 64, ti = r / G, h = r % G;
       if (ti < nr) {
-        const size_t head = ((size_t)row_win + pw[p0 + ti]) * hq + (size_t)g * G + h;
+        const size_t head = ((size_t)row_win + tok_off(ti)) * hq + (size_t)g * G + h;
         for (int c = 0; c < kD; ++c)
           out[head * kD + c] = __float2bfloat16_rn(gate_apply<bf16>(gate, head, c, kD, 0.f));
         if (lse) lse[head] = -INFINITY;
@@ -420,7 +434,7 @@ __global__ void __launch_bounds__(192, 1) prefill_tc_kernel(
           break;
         }
         const int j = ent[e].x;
-        int pg = page_table[(size_t)b * max_blocks + j];
+        int pg = MSA_IN_BOUNDS(j, max_blocks, status) ? page_table[(size_t)b * max_blocks + j] : 0;
         if (pg < 0 || pg >= num_pages) {
           report(status, MSA_DEV_BAD_PAGE);
           pg = 0;  // keep the pipeline in step; the result of this unit is unspecified
@@ -490,7 +504,7 @@ __global__ void __launch_bounds__(192, 1) prefill_tc_kernel(
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
     const int ti = r / G, h = r % G;               // token within the tile, head in the group
     const bool row_ok = ti < nr;
-    const int o_tok = row_ok ? pw[p0 + ti] : 0;    // the token's offset in its window
+    const int o_tok = row_ok ? tok_off(ti) : 0;    // the token's offset in its window
     const int t = t_win + o_tok;                   // position of this row's token
     const size_t qrow = (size_t)row_win + o_tok;   // its global query row
     // Q row -> TMEM (bf16 pairs as 32-bit columns)
@@ -537,7 +551,7 @@ __global__ void __launch_bounds__(192, 1) prefill_tc_kernel(
     for (int hv = 0; hv < 2; ++hv) {
       ti_half[hv] = (quarter * 32 + hv * 16 + (lane & 15)) / G;
       ok_half[hv] = ti_half[hv] < nr;
-      t_half[hv] = t_win + (ok_half[hv] ? pw[p0 + ti_half[hv]] : 0);
+      t_half[hv] = t_win + (ok_half[hv] ? tok_off(ti_half[hv]) : 0);
     }
     const bool upper = lane >= 16;  // which 64 columns of the half-mode row
     int2 en_next = ent[0];

@@ -87,6 +87,12 @@ __device__ __forceinline__ void load_qbar_vec(const T* __restrict__ qrow, int G,
   for (int x = 0; x < VEC; ++x) out[x] = acc[x];
 }
 
+__device__ __forceinline__ uint64_t shfl_xor_u64(uint64_t v, int m) {
+  const uint32_t lo = __shfl_xor_sync(0xffffffffu, (uint32_t)v, m);
+  const uint32_t hi = __shfl_xor_sync(0xffffffffu, (uint32_t)(v >> 32), m);
+  return ((uint64_t)hi << 32) | lo;
+}
+
 // Sorted insertion into a descending list of N keys (L[N-1] smallest).
 template <int N>
 __device__ __forceinline__ void insert_key(uint64_t (&L)[N], uint64_t key) {
@@ -148,6 +154,9 @@ __global__ void __launch_bounds__(256, KMAX <= 16 ? 3 : 1) select_rows_kernel(
   const int row0 = cu_q[b];
   const int n_rows = cu_q[b + 1] - row0;
   const int r_lo = blockIdx.x * kRows;
+  // the sequence's rows lie inside q / idx, and the grid covers all of them
+  if (blockIdx.x == 0 && threadIdx.x == 0) (void)MSA_RANGE_OK(n_rows, n_rows, gridDim.x * kRows, status);
+  if (!MSA_RANGE_OK(row0, row0 + n_rows, cu_q[gridDim.y], status)) return;
   if (r_lo >= n_rows) return;
   const int nr = min(kRows, n_rows - r_lo);
   const int L = seq_lens[b];
@@ -182,6 +191,14 @@ __global__ void __launch_bounds__(256, KMAX <= 16 ? 3 : 1) select_rows_kernel(
   uint64_t top[KMAX];
 #pragma unroll
   for (int s = 0; s < KMAX; ++s) top[s] = 0ull;
+  // Row threshold. The row keeps its best k-1 <= KMAX candidates, and its
+  // SUBS threads hold SUBS * QK = KMAX keys at or above the smallest of their
+  // QK-th best keys. A candidate below that key has k-1 better ones already
+  // and can never be kept, so it is not inserted; every key of the final
+  // selection still reaches its thread's list, and the selection is
+  // unchanged. Refreshed after every chunk (0 until each thread holds QK keys).
+  constexpr int QK = KMAX / SUBS;
+  uint64_t row_thr = 0ull;
 
   // score micro-tile: thread (tr, tc) -> rows 2tr, 2tr+1 and candidates tc + 16m, m < 4
   const int tr = tid / 16, tc = tid % 16;
@@ -241,13 +258,34 @@ __global__ void __launch_bounds__(256, KMAX <= 16 ? 3 : 1) select_rows_kernel(
         for (int m = 0; m < 4; ++m) sc[(2 * tr + a) * kChunk + tc + 16 * m] = acc[a][m];
     }
     __syncthreads();
+    // the chunk's candidates above the thresholds, one bit each, then the
+    // inserts: a warp runs as many insert rounds as its busiest thread has
+    // survivors, not one per candidate
+    uint32_t live = 0u;
     if (sr < nr) {
-      for (int jj = ss; jj < nc; jj += SUBS) {
-        const int j = c0 + jj;
-        if (j >= my_nc || s_page[jj] < 0) continue;
-        insert_key<KMAX>(top, sel_key(sc[sr * kChunk + jj], j));
+      const uint64_t thr = row_thr > top[KMAX - 1] ? row_thr : top[KMAX - 1];
+#pragma unroll
+      for (int m = 0; m < kChunk / SUBS; ++m) {
+        const int jj = ss + m * SUBS, j = c0 + jj;
+        if (jj < nc && j < my_nc && s_page[jj] >= 0 && sel_key(sc[sr * kChunk + jj], j) > thr)
+          live |= 1u << m;
       }
     }
+    while (live) {
+      const int m = __ffs(live) - 1;
+      live &= live - 1u;
+      const int jj = ss + m * SUBS;
+      insert_key<KMAX>(top, sel_key(sc[sr * kChunk + jj], c0 + jj));
+    }
+    // refresh the row threshold: the minimum over the row's SUBS threads (SUBS
+    // consecutive lanes of one warp) of their QK-th best key
+    uint64_t kth = top[QK - 1];
+#pragma unroll
+    for (int o = 1; o < SUBS; o <<= 1) {
+      const uint64_t x = shfl_xor_u64(kth, o);
+      kth = x < kth ? x : kth;
+    }
+    row_thr = kth;
   }
 
   // merge the SUBS lists of each row pairwise (3 levels). Two descending lists
@@ -295,11 +333,6 @@ __global__ void __launch_bounds__(256, KMAX <= 16 ? 3 : 1) select_rows_kernel(
 // ---------------------------------------------------------------------------
 // select_decode
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ uint64_t shfl_xor_u64(uint64_t v, int m) {
-  const uint32_t lo = __shfl_xor_sync(0xffffffffu, (uint32_t)v, m);
-  const uint32_t hi = __shfl_xor_sync(0xffffffffu, (uint32_t)(v >> 32), m);
-  return ((uint64_t)hi << 32) | lo;
-}
 
 // Pass 1 of decode selection. An item is (sequence b, chunk c of 64 candidate
 // blocks, subset gs of hg consecutive KV groups); items are numbered over the
@@ -455,7 +488,8 @@ __global__ void __launch_bounds__(kPass1Threads + 32, 1) select_decode_pass1(
       bool valid = false;
       if (pg != kNoCand) {
         if (pg < 0 || pg >= num_pages) report(status, MSA_DEV_BAD_PAGE);
-        else valid = true;
+        else valid = MSA_RANGE_OK((size_t)lane * pstride, (size_t)lane * pstride + page_bytes,
+                                  stage_bytes, status);
       }
       const uint32_t vb = __ballot_sync(0xffffffffu, valid);
       unsigned char* st = smem_raw + (size_t)s * stage_bytes;
@@ -584,7 +618,7 @@ __global__ void __launch_bounds__(kPass1Threads + 32, 1) select_decode_pass1(
         }
       }
     }
-    if (active) {
+    if (active && MSA_IN_BOUNDS(b, batch, status) && MSA_IN_BOUNDS(c, nchunks, status)) {
       uint64_t* out = ws + (((size_t)b * hkv + gs * hg + my_g) * nchunks + c) * kw;
 #pragma unroll
       for (int r = 0; r < KPL; ++r) {

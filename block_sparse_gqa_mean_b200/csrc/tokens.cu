@@ -93,7 +93,8 @@ __device__ __forceinline__ bool token_row(int r, const int32_t* __restrict__ cu_
   const int n_b = cu_q[lo + 1] - cu_q[lo];
   const int L = seq_lens[lo];
   t = L - n_b + (r - cu_q[lo]);
-  return n_b <= L && L <= max_blocks * B && t >= 0;
+  // r past cu_q[batch] (more rows than the offsets describe) has no position
+  return n_b <= L && L <= max_blocks * B && t >= 0 && r - cu_q[lo] < n_b;
 }
 
 }  // namespace
@@ -167,7 +168,8 @@ __global__ void __launch_bounds__(256) tok_score_kernel(
         if (lane == step * RPI + r) res = v;
       }
     }
-    if (u0 + lane < t) scores[(size_t)r * max_len + u0 + lane] = res;
+    if (u0 + lane < t && MSA_IN_BOUNDS(u0 + lane, max_len, status))
+      scores[(size_t)r * max_len + u0 + lane] = res;
   }
 }
 

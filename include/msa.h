@@ -81,6 +81,9 @@ typedef enum msa_dtype { MSA_DTYPE_BF16 = 0, MSA_DTYPE_F32 = 1 } msa_dtype_t;
 #define MSA_DEV_BAD_LENGTH 0x2u /* length beyond capacity, or rows beyond seq_len   */
 #define MSA_DEV_BAD_INDEX 0x4u  /* block index outside [0, own block] or unsorted   */
 #define MSA_DEV_TIMEOUT 0x8u    /* a bounded device-side wait gave up               */
+#define MSA_DEV_BOUNDS 0x10u    /* bounds-checked build only: an index derived from
+                                   device data or a launch-size assumption fell
+                                   outside its buffer; the access was skipped      */
 
 /* The paged cache, passed by pointer. Host integers size the grids, so no
  * entry point reads device memory on the host. */
@@ -123,7 +126,10 @@ typedef enum msa_op {
  *   k_new, v_new      : device [N_new][num_kv_heads][head_dim], kv->dtype. The
  *                       rows of sequence b are cu_new[b] .. cu_new[b+1]-1.
  *   cu_new            : device [batch+1] int32, non-decreasing, cu_new[0] = 0.
- *   max_new_per_seq   : host bound on cu_new[b+1]-cu_new[b] (sizes the grid).
+ *   max_new_per_seq   : host bound on cu_new[b+1]-cu_new[b] (sizes the grid; a
+ *                       sequence with more new rows is only partly appended,
+ *                       which the bounds-checked build reports as
+ *                       MSA_DEV_BOUNDS).
  *
  * kv->seq_lens must already count the new tokens: sequence b's new rows go to
  * positions seq_lens[b]-n_b .. seq_lens[b]-1. Writes those rows into the pages
@@ -153,7 +159,9 @@ msa_status_t msa_build_block_cache(const msa_paged_kv_t* kv, const void* k_new, 
  *                       LAST n_b positions: seq_lens[b]-n_b .. seq_lens[b]-1.
  *                       NULL means decode: num_rows == batch, row b at
  *                       position seq_lens[b]-1.
- *   max_rows_per_seq  : host bound on n_b (sizes the grid; 1 for decode).
+ *   max_rows_per_seq  : host bound on n_b (sizes the grid; 1 for decode). Rows
+ *                       of a sequence past this bound get no output (the
+ *                       bounds-checked build reports MSA_DEV_BOUNDS).
  *   block_idx         : device out [num_rows][num_kv_heads][top_k] int32, the
  *                       selected logical blocks in ascending order, -1 padded.
  *   block_score       : device out, same shape, fp32, or NULL: the score of
@@ -418,6 +426,22 @@ const char* msa_status_string(msa_status_t status);
 
 /* Library ABI version (major * 1000 + minor). */
 int32_t msa_version(void);
+
+/* How this copy of the library was compiled: a mask of MSA_BUILD_* bits.
+ *  MSA_BUILD_DEBUG_BOUNDS: the bounds-checked build (compiled with
+ *    -DMSA_DEBUG_BOUNDS, shipped as libmsa_debug.so beside libmsa.so). Every
+ *    shared- or global-memory index that a kernel derives from device data
+ *    (cu_q / cu_seqlens entries, block and token indices, plan and order
+ *    tables the library writes itself) or from a launch-size assumption is
+ *    compared with the extent of its buffer before the access; a failed check
+ *    sets MSA_DEV_BOUNDS in *kv->status_word and skips the access (a TMA
+ *    coordinate is replaced by a valid one so that the pipeline stays in
+ *    step) instead of faulting. Outputs are identical to the regular build's
+ *    when no check fails. It is a debugging aid that stands in for a memory
+ *    checker and costs a few percent of speed; the regular build compiles the
+ *    checks to nothing. */
+#define MSA_BUILD_DEBUG_BOUNDS 0x1
+int32_t msa_build_flags(void);
 
 #ifdef __cplusplus
 }
