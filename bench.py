@@ -447,7 +447,7 @@ def run_decode(w, steps, warmup, world, flush_l2):
         raise RuntimeError(f"device status {status:#x}")
     return {"step_ms": per_step[0], "kernel_ms": k_ms, "clocks": clk.summary(),
             "e2e_ms": e2e_ms, "h2d": (hq_.numel() + hk.numel() + hv.numel()) * 2,
-            "d2h": hout.numel() * 2, "launches_per_step": 1 + 2 + 2}
+            "d2h": hout.numel() * 2, "launches_per_step": 1 + 2 + 1}
 
 
 def run_decode_steps(w, world):
@@ -548,7 +548,7 @@ def run_decode_steps(w, world):
     return {"step_ms": sum(step_ms) / S, "step_ms_first_last": [step_ms[0], step_ms[-1]],
             "kernel_ms": k_ms, "clocks": clk.summary(), "e2e_ms": e2e_ms,
             "h2d": (hq_[0].numel() + hk[0].numel() + hv[0].numel()) * 2,
-            "d2h": hout[0].numel() * 2, "launches_per_step": 1 + 2 + 2, "steps": S}
+            "d2h": hout[0].numel() * 2, "launches_per_step": 1 + 2 + 1, "steps": S}
 
 
 TOKEN_HEADS = 32      # indexer heads ("Sparse Attention + Linear Backbones", 5.3: 32 x 128)
@@ -944,7 +944,7 @@ def decode_block(w, args, world, pk):
     traffic = None
     if w.name == "paged_decode_bf16" and w.batch == 32:
         t1 = profile_traffic("select_decode_pass1", "select.cu")
-        t2 = profile_traffic("decode_splitk_kernel", "decode_splitk.cu")
+        t2 = profile_traffic("decode_streamk_kernel", "decode_splitk.cu")
         traffic = t1 + t2 if t1 is not None and t2 is not None else None
     return {"workload": w.name, "value": w.batch * world / (ms * 1e-3), "unit": "tokens/s",
             "ms_per_step": ms, "hbm_gbs": nbytes / (ms * 1e-3) / 1e9,
@@ -952,7 +952,7 @@ def decode_block(w, args, world, pk):
                          "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": nbytes / (ms * 1e-3) / 1e9 / pk["hbm_gbs"],
                          "traffic": traffic,
-                         "traffic_scope": "select_decode_pass1 + decode_splitk_kernel DRAM bytes",
+                         "traffic_scope": "select_decode_pass1 + decode_streamk_kernel DRAM bytes",
                          "peak_source": f"{pk['source']} HBM copy",
                          "scope": "whole decode step (append+select+attention)",
                          "algorithmic_bytes_per_step": nbytes,

@@ -8,11 +8,15 @@
 // writes must stay consistent with the index. Here every write of a token
 // re-pools the centroid of the block it lands in, in the same kernel.
 //
-// One CTA per (sequence, touched block, KV head). It copies the new rows of
-// that block into the page (16-byte vector copies), stages the block's keys
-// in shared memory, then every thread owns one coordinate and sums the keys
-// present in the block in token order, in fp32, and divides by the count. The order does not depend on how the tokens
-// arrived, so token-by-token appends and a one-shot build give equal bits.
+// One CTA per (sequence, touched block, KV head). It stages the block's keys
+// in shared memory - the rows already in the page and the new rows from the
+// input are loaded together, 16-byte vectors, up to 16 per thread in flight,
+// so a decode step's append costs one memory latency, not a store followed
+// by a reload - writes the new key and value rows into the page, then every
+// thread owns one coordinate and sums the keys present in the block in token
+// order, in fp32, and divides by the count. The order does not depend on how
+// the tokens arrived, so token-by-token appends and a one-shot build give
+// equal bits.
 #include "common.cuh"
 
 namespace msa {
@@ -51,32 +55,59 @@ __global__ void __launch_bounds__(128) append_pool_kernel(
   const int u_lo = max(t0, j * B);
   const int u_hi = min(L, (j + 1) * B);
   const size_t page_off = ((size_t)page * hkv + g) * B * D;
+  const size_t pool = (size_t)num_pages * hkv * B * D;
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  T* tile = reinterpret_cast<T*>(smem_raw);  // [n][D]
 
-  // 1) copy the new rows of this block: 16-byte chunks, D/8 (bf16) or D/4 (fp32) per row
+  // 1) the block's keys into shared memory, the new ones also into the page;
+  //    the new values into the page. 16-byte chunks, CPR per row.
   constexpr int VEC = 16 / sizeof(T);
-  constexpr int CPR = D / VEC;  // chunks per row
-  const int nrows = u_hi - u_lo;
-  for (int c = threadIdx.x; c < nrows * CPR; c += blockDim.x) {
+  constexpr int CPR = D / VEC;
+  constexpr int NV = 16;                 // chunks in flight per thread
+  const int n = u_hi - j * B;            // tokens in the block after the append
+  const int total = n * CPR;
+  const int first_new = (u_lo - j * B) * CPR;  // chunks before this one are in the page already
+  auto new_src = [&](int c) {  // offset in k_new / v_new of chunk c of a new row
     const int r = c / CPR, col = (c % CPR) * VEC;
-    const int u = u_lo + r;
-    const size_t src = ((size_t)(row0 + (u - t0)) * hkv + g) * D + col;
-    const size_t dst = page_off + (size_t)(u - j * B) * D + col;
-    if (!MSA_RANGE_OK(dst, dst + VEC, (size_t)num_pages * hkv * B * D, status)) continue;
-    *reinterpret_cast<uint4*>(k_pages + dst) = *reinterpret_cast<const uint4*>(k_new + src);
-    *reinterpret_cast<uint4*>(v_pages + dst) = *reinterpret_cast<const uint4*>(v_new + src);
+    return ((size_t)(row0 + (j * B + r - t0)) * hkv + g) * D + col;
+  };
+  // this thread's first value chunk is loaded before the keys, so its latency
+  // overlaps theirs (a decode step has one new row: one chunk per thread at most)
+  const int vc0 = first_new + (int)threadIdx.x;
+  uint4 v_first = make_uint4(0u, 0u, 0u, 0u);
+  if (vc0 < total) v_first = *reinterpret_cast<const uint4*>(v_new + new_src(vc0));
+  for (int base = 0; base < total; base += NV * 128) {
+    uint4 kv4[NV];
+#pragma unroll
+    for (int x = 0; x < NV; ++x) {
+      const int c = base + x * 128 + (int)threadIdx.x;
+      if (c < total) {
+        if (c < first_new) {
+          kv4[x] = reinterpret_cast<const uint4*>(k_pages + page_off)[c];
+        } else {
+          kv4[x] = *reinterpret_cast<const uint4*>(k_new + new_src(c));
+        }
+      }
+    }
+#pragma unroll
+    for (int x = 0; x < NV; ++x) {
+      const int c = base + x * 128 + (int)threadIdx.x;
+      if (c < total && MSA_IN_BOUNDS(c, B * CPR, status)) {
+        reinterpret_cast<uint4*>(tile)[c] = kv4[x];
+        const size_t dst = page_off + (size_t)c * VEC;
+        if (c >= first_new && MSA_RANGE_OK(dst, dst + VEC, pool, status))
+          *reinterpret_cast<uint4*>(k_pages + dst) = kv4[x];
+      }
+    }
+  }
+  for (int c = vc0; c < total; c += blockDim.x) {
+    const size_t dst = page_off + (size_t)c * VEC;
+    const uint4 v = c == vc0 ? v_first : *reinterpret_cast<const uint4*>(v_new + new_src(c));
+    if (MSA_RANGE_OK(dst, dst + VEC, pool, status)) *reinterpret_cast<uint4*>(v_pages + dst) = v;
   }
   __syncthreads();
 
-  // 2) re-pool the block: mean over every token present, fixed token order.
-  //    The block's keys are staged in shared memory with 16-byte loads first.
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  T* tile = reinterpret_cast<T*>(smem_raw);  // [n][D]
-  const int n = u_hi - j * B;
-  for (int c = threadIdx.x; c < n * CPR; c += blockDim.x)
-    if (MSA_IN_BOUNDS(c, B * CPR, status))
-      reinterpret_cast<uint4*>(tile)[c] =
-          reinterpret_cast<const uint4*>(k_pages + page_off)[c];
-  __syncthreads();
+  // 2) re-pool the block: mean over every token present, fixed token order
   for (int i = threadIdx.x; i < D; i += blockDim.x) {
     float s = 0.f;
     for (int u = 0; u < n; ++u) s = __fadd_rn(s, to_f32(tile[u * D + i]));

@@ -1,24 +1,26 @@
-// Allocation-free decode attention: msa_sparse_attn_decode with its split-k
-// scratch in a fixed device array owned by the library.
+// Allocation-free decode attention: msa_sparse_attn_decode with its scratch
+// (one attention part and one flag per resident CTA) in a fixed device array
+// owned by the library.
 //
 // Who needs this: callers that cannot allocate device memory at the point of
 // the call - for instance a plugin invoked from a host framework that owns the
 // whole device memory pool and gives its plugins no scratch allocator, or a
 // latency-critical loop that must not touch the allocator (cudaMalloc can
 // synchronise the device). They pass only inputs and outputs; the partial
-// results of the split-k pass live in g_decode_scratch below.
+// results of the attention kernel live in g_decode_scratch below.
 //
 // Costs and rules of use:
 //  * the array is kNoAllocScratchBytes (8 MiB) of device memory that every
 //    GPU which loads libmsa.so holds until the process exits;
-//  * problems whose split-k partials need more than that
-//    (msa_workspace_size(MSA_OP_DECODE, ...) > 8 MiB) are rejected with
+//  * the decode workspace is bounded by the resident grid, not the batch
+//    (under 5 MiB on 148 SMs at 16 query heads per group), so every supported
+//    shape fits; a problem that needed more than 8 MiB would be rejected with
 //    MSA_ERR_WORKSPACE before anything is launched;
 //  * all calls on a device share the one array, so two calls whose kernels
 //    overlap on the GPU (different streams without ordering between them)
-//    race on it; calls on one stream are safe. Every partial a call reads is
-//    written by the same call first, so nothing has to start at zero and the
-//    contents left by the previous call do not matter;
+//    race on it; calls on one stream are safe. A part is read only after its
+//    flag carries the reading call's own tag, so nothing has to start at zero
+//    and the contents left by the previous call do not matter;
 //  * the first call on each device looks up the array's device address with
 //    cudaGetSymbolAddress (the host-side name of a __device__ array is not a
 //    device address); make that first call before any stream capture.

@@ -105,26 +105,26 @@ __device__ __forceinline__ void insert_key(uint64_t (&L)[N], uint64_t key) {
   L[0] = key > L[0] ? key : L[0];
 }
 
-// Write the selection of one (row, group): `n` chosen past blocks given as
-// keys (any order, 0 = empty), plus the own block, ascending, -1 padded.
-__device__ void write_selection(const uint64_t* keys, int n, int own, int top_k, int32_t* idx_out,
-                                float* score_out) {
+// Write the selection of one (row, group) from the `lanes` threads that
+// share it (consecutive lanes of one warp, `part` = this thread's index among
+// them): `keys` holds the chosen past blocks, descending, non-zero keys first
+// (a zero key is an empty slot). Output: those blocks ascending, then the own
+// block, then -1. Each thread ranks keys part, part + lanes, ... by counting
+// the keys with a lower block index.
+__device__ void write_selection(const uint64_t* keys, int n, int own, int top_k, int part,
+                                int lanes, int32_t* idx_out, float* score_out) {
   int cnt = 0;
-  for (int a = 0; a < n; ++a) cnt += keys[a] != 0ull;
-  for (int a = 0; a < n; ++a) {
-    if (keys[a] == 0ull) continue;
+  while (cnt < n && keys[cnt] != 0ull) ++cnt;
+  for (int a = part; a < cnt; a += lanes) {
     const int ja = key_block(keys[a]);
     int rank = 0;
-    for (int c = 0; c < n; ++c)
-      if (keys[c] != 0ull && key_block(keys[c]) < ja) ++rank;
+    for (int c = 0; c < cnt; ++c) rank += key_block(keys[c]) < ja;
     idx_out[rank] = ja;
     if (score_out) score_out[rank] = key_score(keys[a]);
   }
-  idx_out[cnt] = own;
-  if (score_out) score_out[cnt] = __int_as_float(0x7f800000);
-  for (int s = cnt + 1; s < top_k; ++s) {
-    idx_out[s] = -1;
-    if (score_out) score_out[s] = __int_as_float(0xff800000);
+  for (int s = cnt + part; s < top_k; s += lanes) {
+    idx_out[s] = s == cnt ? own : -1;
+    if (score_out) score_out[s] = __int_as_float(s == cnt ? 0x7f800000 : 0xff800000);
   }
 }
 
@@ -321,12 +321,16 @@ __global__ void __launch_bounds__(256, KMAX <= 16 ? 3 : 1) select_rows_kernel(
     }
     __syncthreads();
   }
+  const int keep = min(top_k - 1, my_nc);
   if (ss == 0 && sr < nr) {
-    const int keep = min(top_k - 1, my_nc);
 #pragma unroll
     for (int s = 0; s < KMAX; ++s) my_list[s] = (s < keep) ? top[s] : 0ull;
+  }
+  __syncwarp();  // the row's SUBS threads are consecutive lanes of one warp
+  if (sr < nr) {
     const size_t out = ((size_t)(row0 + r_lo + sr) * hkv + g) * top_k;
-    write_selection(my_list, min(keep, KMAX), my_t / B, top_k, idx + out, score ? score + out : nullptr);
+    write_selection(lists + (size_t)sr * SUBS * KMAX, min(keep, KMAX), my_t / B, top_k, ss, SUBS,
+                    idx + out, score ? score + out : nullptr);
   }
 }
 

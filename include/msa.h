@@ -207,8 +207,10 @@ msa_status_t msa_sparse_attn_prefill(const msa_paged_kv_t* kv, const void* q, co
 
 /*
  * msa_sparse_attn_decode - the same attention for one new query per sequence
- * (position seq_lens[b]-1, its own token already appended), computed as
- * split-k partials over the selected blocks and merged by log-sum-exp.
+ * (position seq_lens[b]-1, its own token already appended). One kernel: the
+ * selection slots of all sequences and groups are split evenly over one wave
+ * of resident CTAs; a (sequence, group) split over several CTAs is finished,
+ * by log-sum-exp, by the CTA that holds its first blocks.
  *
  * Follows "Art of Focus: Ling 2.0 ...", "Summarizing the Breakthrough" (during
  * decode only the top-k relevant blocks are fetched) and the attention rule
@@ -219,7 +221,11 @@ msa_status_t msa_sparse_attn_prefill(const msa_paged_kv_t* kv, const void* q, co
  *                       rules as for prefill (ascending, -1 padded, an
  *                       adjacent repeat counts once, an empty row gives 0).
  *   out, lse          : device [batch][num_q_heads][head_dim] / [batch][num_q_heads].
- *   workspace         : device scratch, msa_workspace_size(MSA_OP_DECODE, ..).
+ *   workspace         : device scratch, msa_workspace_size(MSA_OP_DECODE, ..):
+ *                       one part per resident CTA (about 4 * SMs * G * 516
+ *                       bytes, whatever the batch) and its flag. Its content
+ *                       on entry does not matter; concurrent calls need
+ *                       separate workspaces.
  */
 msa_status_t msa_sparse_attn_decode(const msa_paged_kv_t* kv, const void* q,
                                     const int32_t* block_idx, int32_t top_k, float softmax_scale,
@@ -275,13 +281,14 @@ msa_status_t msa_sparse_attn_decode_gated(const msa_paged_kv_t* kv, const void* 
  * such call; it exists for those callers only.
  *
  * Same arguments and results as msa_sparse_attn_decode minus the workspace:
- * the split-k partials go to one 8 MiB device array inside libmsa.so, which
- * every GPU that loads the library keeps until the process exits.
+ * the per-CTA parts and flags go to one 8 MiB device array inside libmsa.so,
+ * which every GPU that loads the library keeps until the process exits.
  *  - Bad arguments give the same status as msa_sparse_attn_decode, checked
  *    before anything else (the array is not looked up).
- *  - Returns MSA_ERR_WORKSPACE, launching nothing, when the problem needs more
- *    than 8 MiB, i.e. when msa_workspace_size(MSA_OP_DECODE, kv, batch, 1,
- *    top_k) > 8 MiB (about batch * num_q_heads * splits * 516 bytes).
+ *  - The decode workspace does not grow with the batch (at most about
+ *    4 * SMs * 16 * 516 bytes, under 5 MiB on 148 SMs), so every supported
+ *    shape fits; MSA_ERR_WORKSPACE (nothing launched) is returned only if
+ *    msa_workspace_size(MSA_OP_DECODE, ...) ever exceeded 8 MiB.
  *  - All calls on a device share the array: calls whose kernels may overlap
  *    on the GPU (unordered streams) race; calls on one stream do not. Nothing
  *    in the array needs to start at zero.
