@@ -14,11 +14,14 @@
 //   tok_score_kernel   one score per earlier position (indexer keys are paged
 //                      with the KV cache's page table, one row per position),
 //                      read as whole rows by half-warps
-//   tok_select_kernel  one CTA per sequence: radix select of the (K-1)-th
-//                      largest score on order-preserving 32-bit keys (four
-//                      8-bit passes), then an ordered compaction that keeps
-//                      every larger key and the lowest positions among the
-//                      equal ones, so the list comes out ascending
+//   tok_select_kernel  one CTA per row: radix select of the (K-1)-th largest
+//                      score on order-preserving 32-bit keys (four 8-bit
+//                      passes), then an ordered compaction that keeps every
+//                      larger key and the lowest positions among the equal
+//                      ones, so the list comes out ascending. Long rows first
+//                      narrow the keys to the candidates above a threshold
+//                      read off a sorted regular sample and run both steps on
+//                      those alone, in shared memory
 //   tok_attn_tc_kernel one CTA per (sequence, KV group) for bf16, head_dim 128:
 //                      the kept tokens' K and V rows gathered 64 at a time by
 //                      16-byte cp.async copies into a three-stage ring of
@@ -36,6 +39,7 @@ constexpr int kScoreChunk = 1024;  // positions per score CTA (256 threads x 4)
 constexpr int kSelThreads = 1024;
 constexpr int kSelWarps = kSelThreads / 32;
 constexpr int kTokChunk = 32;      // tokens gathered per attention step
+constexpr int kCandCap = 16384;    // candidates of the sampled selection (keys + positions: 128 KB)
 
 __device__ __forceinline__ unsigned order_key(float f) {
   const unsigned b = __float_as_uint(f);
@@ -70,6 +74,41 @@ __device__ __forceinline__ unsigned block_scan_1024(unsigned v, unsigned* warp_t
   *total = warp_tot[32];
   __syncthreads();
   return r;
+}
+
+// Warp 0 of a radix-select pass: walking the 256 bins of `hist` from the top,
+// the digit d at which the count reaches `remaining`, and the count of the
+// bins above d (bin 0 when the bins never reach it). Lane l holds bins
+// 255 - 8l down to 248 - 8l.
+__device__ __forceinline__ void pick_digit(const unsigned* hist, unsigned remaining, unsigned* s_d,
+                                           unsigned* s_cum) {
+  const int lane = threadIdx.x & 31;
+  unsigned v[8], sum = 0u;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    v[i] = hist[255 - 8 * lane - i];
+    sum += v[i];
+  }
+  unsigned incl = sum;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned x = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += x;
+  }
+  const unsigned reach = __ballot_sync(0xffffffffu, incl >= remaining);
+  const int at = reach ? __ffs(reach) - 1 : 31;
+  if (lane == at) {
+    unsigned cum = incl - sum;
+    int d = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      d = 255 - 8 * lane - i;
+      if (cum + v[i] >= remaining || d == 0) break;
+      cum += v[i];
+    }
+    *s_d = (unsigned)d;
+    *s_cum = cum;
+  }
 }
 
 // Row r of a token-variant call: its sequence b and position t. Without cu_q
@@ -195,6 +234,134 @@ __global__ void __launch_bounds__(kSelThreads) tok_select_kernel(
     return;
   }
   const float* sc = scores + (size_t)r * max_len;
+
+  // Sampled selection (long rows, keep <= kCandCap / 4). A regular sample of
+  // kSelThreads scores, sorted, gives a key tau that about (rk / kSelThreads)
+  // of all keys reach, rk set to 1.5 x the sample rank of the keep-th largest
+  // plus 16; every key >= tau is a candidate. When the candidates number at
+  // least keep (so the keep largest are among them) and fit in shared memory,
+  // the selection below runs on them alone, in position order; otherwise the
+  // full radix select further down runs. Either way the result is the exact
+  // rule: the keep largest keys, ties to the lower position.
+  if (keep <= kCandCap / 4 && n >= 8 * kSelThreads) {
+    extern __shared__ __align__(16) unsigned char cand_smem[];
+    unsigned* c_key = reinterpret_cast<unsigned*>(cand_smem);  // [kCandCap]
+    int* c_pos = reinterpret_cast<int*>(c_key + kCandCap);      // [kCandCap]
+    unsigned* samp = whist;                                     // [kSelThreads], reused
+    samp[tid] = order_key(sc[(long long)tid * n / kSelThreads]);
+    __syncthreads();
+    for (int size = 2; size <= kSelThreads; size <<= 1) {  // bitonic sort, descending
+      for (int stride = size >> 1; stride > 0; stride >>= 1) {
+        const int p = tid ^ stride;
+        if (p > tid) {
+          const unsigned a = samp[tid], c = samp[p];
+          if (((tid & size) == 0) ? a < c : a > c) {
+            samp[tid] = c;
+            samp[p] = a;
+          }
+        }
+        __syncthreads();
+      }
+    }
+    const long long srank = ((long long)keep * kSelThreads + n - 1) / n;
+    const unsigned tau = samp[(int)min((long long)kSelThreads - 1, srank + srank / 2 + 16)];
+    // each thread a contiguous, 16-byte aligned run of positions, 8 vectors in flight
+    const int per = (((n + kSelThreads - 1) / kSelThreads) + 3) & ~3;
+    const int a0 = min(n, tid * per), a1 = min(n, a0 + per);
+    unsigned cnt = 0u;
+    for (int u = a0; u < a1; u += 32) {
+      float4 f[8];
+#pragma unroll
+      for (int x = 0; x < 8; ++x)
+        if (u + 4 * x < a1) f[x] = *reinterpret_cast<const float4*>(sc + u + 4 * x);
+#pragma unroll
+      for (int x = 0; x < 8; ++x) {
+        const float fv[4] = {f[x].x, f[x].y, f[x].z, f[x].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          cnt += (u + 4 * x + e < a1 && order_key(fv[e]) >= tau) ? 1u : 0u;
+      }
+    }
+    unsigned total;
+    unsigned w = block_scan_1024(cnt, warp_tot, &total);
+    if (total >= (unsigned)keep && total <= (unsigned)kCandCap) {  // the same in every thread
+      for (int u = a0; u < a1; u += 32) {
+        float4 f[8];
+#pragma unroll
+        for (int x = 0; x < 8; ++x)
+          if (u + 4 * x < a1) f[x] = *reinterpret_cast<const float4*>(sc + u + 4 * x);
+#pragma unroll
+        for (int x = 0; x < 8; ++x) {
+          const float fv[4] = {f[x].x, f[x].y, f[x].z, f[x].w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const unsigned k = order_key(fv[e]);
+            if (u + 4 * x + e < a1 && k >= tau && MSA_IN_BOUNDS(w, kCandCap, nullptr)) {
+              c_key[w] = k;
+              c_pos[w] = u + 4 * x + e;
+              ++w;
+            }
+          }
+        }
+      }
+      __syncthreads();
+      // radix select of the keep-th largest candidate key
+      unsigned prefix = 0u, pmask = 0u, remaining = (unsigned)keep;
+      for (int shift = 24; shift >= 0; shift -= 8) {
+        for (int i = tid; i < 256 * kSelWarps; i += kSelThreads) whist[i] = 0u;
+        __syncthreads();
+        unsigned* wh = whist + (tid / 32) * 256;
+        for (int i = tid; i < (int)total; i += kSelThreads) {
+          const unsigned k = c_key[i];
+          if ((k & pmask) == prefix) atomicAdd(&wh[(k >> shift) & 255u], 1u);
+        }
+        __syncthreads();
+        for (int i = tid; i < 256; i += kSelThreads) {
+          unsigned c = 0u;
+          for (int ww = 0; ww < kSelWarps; ++ww) c += whist[ww * 256 + i];
+          hist[i] = c;
+        }
+        __syncthreads();
+        if (tid < 32) pick_digit(hist, remaining, &s_prefix, &s_remaining);
+        __syncthreads();
+        prefix |= s_prefix << shift;
+        remaining -= s_remaining;
+        pmask |= 255u << shift;
+        __syncthreads();
+      }
+      const unsigned T_key = prefix;
+      // ordered selection over the candidates (already in position order)
+      const int cper = ((int)total + kSelThreads - 1) / kSelThreads;
+      const int c0 = min((int)total, tid * cper), c1 = min((int)total, c0 + cper);
+      unsigned eq = 0u;
+      for (int i = c0; i < c1; ++i) eq += c_key[i] == T_key;
+      unsigned tot;
+      const unsigned eq_before = block_scan_1024(eq, warp_tot, &tot);
+      unsigned sel = 0u;
+      {
+        unsigned e2 = eq_before;
+        for (int i = c0; i < c1; ++i) {
+          const unsigned k = c_key[i];
+          sel += (k > T_key || (k == T_key && e2 < remaining)) ? 1u : 0u;
+          e2 += k == T_key;
+        }
+      }
+      unsigned pos = block_scan_1024(sel, warp_tot, &tot);
+      {
+        unsigned e2 = eq_before;
+        for (int i = c0; i < c1; ++i) {
+          const unsigned k = c_key[i];
+          const bool s2 = k > T_key || (k == T_key && e2 < remaining);
+          e2 += k == T_key;
+          if (s2 && pos < (unsigned)keep) out[pos++] = c_pos[i];
+        }
+      }
+      for (int i = keep + tid; i < top_k; i += kSelThreads) out[i] = (i == keep) ? t : -1;
+      return;
+    }
+    __syncthreads();  // the sample buffer is reused by the full select
+  }
+
   // radix select: the key of the keep-th largest score, and how many keys equal
   // to it are kept (the lowest positions among them)
   unsigned prefix = 0u, pmask = 0u, remaining = (unsigned)keep;
@@ -228,19 +395,10 @@ __global__ void __launch_bounds__(kSelThreads) tok_select_kernel(
       hist[i] = c;
     }
     __syncthreads();
-    if (tid == 0) {
-      unsigned cum = 0u;
-      int d = 255;
-      for (; d > 0; --d) {
-        if (cum + hist[d] >= remaining) break;
-        cum += hist[d];
-      }
-      s_prefix = prefix | ((unsigned)d << shift);
-      s_remaining = remaining - cum;
-    }
+    if (tid < 32) pick_digit(hist, remaining, &s_prefix, &s_remaining);
     __syncthreads();
-    prefix = s_prefix;
-    remaining = s_remaining;
+    prefix |= s_prefix << shift;
+    remaining -= s_remaining;
     pmask |= 255u << shift;
     __syncthreads();
   }
@@ -634,9 +792,12 @@ static cudaError_t launch_tok_select(const msa_paged_kv_t* kv, const void* ki_pa
                                                kv->max_blocks_per_seq, max_len, scores);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  tok_select_kernel<<<rows, kSelThreads, 0, st>>>(scores, kv->seq_lens, cu_q, kv->batch,
-                                                  kv->max_blocks_per_seq, kv->block_size, max_len,
-                                                  top_k, tok_idx);
+  const size_t cand = (size_t)kCandCap * 8;
+  e = cudaFuncSetAttribute(tok_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)cand);
+  if (e != cudaSuccess) return e;
+  tok_select_kernel<<<rows, kSelThreads, cand, st>>>(scores, kv->seq_lens, cu_q, kv->batch,
+                                                     kv->max_blocks_per_seq, kv->block_size,
+                                                     max_len, top_k, tok_idx);
   return cudaGetLastError();
 }
 

@@ -91,6 +91,81 @@ def test_token_decode_selection_and_attention(top_k):
     compare(out, np.concatenate(refs), w.dtype)
 
 
+def _kept_from_scores(scores, L, top_k):
+    """The selection rule on given fp32 scores of positions 0 .. L-2: the
+    top_k - 1 largest (ties to the lower position), ascending, then L - 1."""
+    n = L - 1
+    keep = min(top_k - 1, n)
+    order = np.lexsort((np.arange(n), -scores[:n].astype(np.float64)))
+    return sorted(order[:keep].tolist()) + [L - 1]
+
+
+# long rows (>= 8192 earlier positions, top_k - 1 <= 4096) take the sampled
+# selection; their oracle gap at top_k 64 is >= GAP_MIN on every row
+LONG_CTX = (9000, 20000, 40000)
+
+
+@pytest.mark.parametrize("top_k", [64, 2048])
+def test_token_decode_long_rows(top_k):
+    w = workloads.paged_decode_bf16(batch=3, ctx=LONG_CTX)
+    p = workloads.paging(w)
+    cache = new_cache(w, p)
+    lens = fill_context(cache, w)
+    after = [L + 1 for L in lens]
+    append(cache, w, lens, after)
+    ki = _index_pages(w, p, after)
+    qi = workloads.indexer_queries(w, 0, HI, DEV)
+    ws = torch.empty(msa.workspace_size(msa.MSA_OP_SELECT_TOKENS, cache, w.batch, 1, top_k),
+                     dtype=torch.uint8, device=DEV)
+    idx = msa.select_tokens(cache, ki, qi, top_k, workspace=ws)
+    torch.cuda.synchronize()
+    assert cache.device_status() == 0
+    gi = idx.cpu().numpy()
+    # the kernel's own fp32 scores, one row of max_blocks * block_size per sequence
+    sc = ws.view(torch.float32)[:w.batch * p.max_blocks * w.block].view(w.batch, -1).cpu().numpy()
+    protected = 0
+    for b in range(w.batch):
+        L = after[b]
+        row = gi[b]
+        kept = [int(u) for u in row if u >= 0]
+        # exact: the rule applied to the scores the kernel computed
+        assert kept == _kept_from_scores(sc[b], L, top_k)
+        assert np.all(row[len(kept):] == -1)
+        # against the oracle (fp64 scores)
+        pos = np.array([L - 1])
+        S = oracle.token_scores(qi[b:b + 1].cpu(), workloads.indexer_keys(w, b, 0, L), pos)
+        oidx, gap = oracle.token_select(S, pos, top_k)
+        if gap[0] >= GAP_MIN:
+            protected += 1
+            assert np.array_equal(row, oidx[0])
+        else:
+            earlier = kept[:-1]
+            cut = np.sort(S[0, :L - 1])[::-1][len(earlier) - 1]
+            assert all(S[0, u] >= cut - 1e-3 for u in earlier)
+    assert protected == (3 if top_k == 64 else 0)
+
+
+@pytest.mark.parametrize("ctx", [(12000,), (20000,)])
+def test_token_decode_all_ties(ctx):
+    """Zero indexer keys: every earlier position scores 0, and the lowest
+    top_k - 1 positions are kept. 12000 positions fit the sampled selection's
+    candidate buffer (ties resolved there), 20000 do not (the full select)."""
+    top_k = 2048
+    w = workloads.paged_decode_bf16(batch=1, ctx=ctx)
+    p = workloads.paging(w)
+    cache = new_cache(w, p)
+    lens = fill_context(cache, w)
+    after = [L + 1 for L in lens]
+    append(cache, w, lens, after)
+    ki = torch.zeros(p.num_pages, w.block, w.d, dtype=w.torch_dtype, device=DEV)
+    qi = workloads.indexer_queries(w, 0, HI, DEV)
+    idx = msa.select_tokens(cache, ki, qi, top_k)
+    torch.cuda.synchronize()
+    assert cache.device_status() == 0
+    expect = list(range(top_k - 1)) + [after[0] - 1]
+    assert idx[0].cpu().tolist() == expect
+
+
 def test_token_decode_repeated_and_empty_lists():
     w = workloads.paged_decode_bf16(batch=2, ctx=(2000, 2500))
     p = workloads.paging(w)
