@@ -446,3 +446,54 @@ def test_device_status_on_bad_page_and_length():
     msa.sparse_attn_decode(cache, q, idx)
     torch.cuda.synchronize()
     assert cache.device_status() == 0
+
+
+def _bits(t):
+    return t.view(torch.int16) if t.dtype == torch.bfloat16 else t.view(torch.int32)
+
+
+@pytest.mark.parametrize("name,make", [
+    ("paged_g4", lambda: workloads.paged_decode_bf16(batch=4, ctx=(3000, 4095, 4096, 5000))),
+    ("long_g8_b128", lambda: workloads.decode_1m_bf16(ctx=(40000,), steps=1)),
+], ids=["paged_g4", "long_g8_b128"])
+def test_decode_graph_replays_and_shared_workspace(name, make):
+    """The decode attention publishes the parts of split (sequence, group) units
+    under a tag drawn per host call, which a CUDA graph captures once, and the
+    finishing CTA clears the flags it read. Replays of one graph, and two graphs
+    (two tags) alternating on one workspace, must give the eager call's bits."""
+    w = make()
+    p = workloads.paging(w)
+    cache = new_cache(w, p)
+    lens = fill_context(cache, w)
+    after = [L + 1 for L in lens]
+    append(cache, w, lens, after)
+    q0 = workloads.queries_decode(w, 0, DEV)
+    q1 = (q0.float() * 0.5).to(q0.dtype)
+    ws = torch.empty(msa.workspace_size(msa.MSA_OP_DECODE, cache, w.batch, 1, w.top_k),
+                     dtype=torch.uint8, device=DEV)
+    idx0, _ = msa.select_topk(cache, q0, w.top_k)
+    idx1, _ = msa.select_topk(cache, q1, w.top_k)
+    ref0, lse0 = msa.sparse_attn_decode(cache, q0, idx0, workspace=ws)
+    ref1, lse1 = msa.sparse_attn_decode(cache, q1, idx1, workspace=ws)
+    torch.cuda.synchronize()
+    out0, l0 = torch.empty_like(ref0), torch.empty_like(lse0)
+    out1, l1 = torch.empty_like(ref1), torch.empty_like(lse1)
+    graphs = []
+    for q, idx, o, l in ((q0, idx0, out0, l0), (q1, idx1, out1, l1)):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            msa.sparse_attn_decode(cache, q, idx, out=o, lse=l, workspace=ws)
+        graphs.append(g)
+    torch.cuda.synchronize()
+    for rep in range(3):
+        for g, o, l, ro, rl in ((graphs[0], out0, l0, ref0, lse0), (graphs[1], out1, l1, ref1, lse1)):
+            o.fill_(float("nan"))
+            g.replay()
+            torch.cuda.synchronize()
+            assert torch.equal(_bits(o), _bits(ro)), (name, rep)
+            assert torch.equal(_bits(l), _bits(rl)), (name, rep)
+    for rep in range(2):  # one graph replayed back to back
+        graphs[0].replay()
+    torch.cuda.synchronize()
+    assert torch.equal(_bits(out0), _bits(ref0))
+    assert cache.device_status() == 0
