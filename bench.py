@@ -8,7 +8,7 @@ A step is one pass of the whole hot path over one batch of synthetic input:
                       top-k selection (msa_select_topk) and sparse attention
                       (msa_sparse_attn_prefill) over all query rows;
   decode workloads  : append of one token per sequence, decode selection and
-                      split-k decode attention.
+                      the stream-K decode attention.
 The default workload is the prefill one (batch 1, 32768 tokens, 32/4 heads,
 d 128, block 128, top-k 16); the other four workloads are measured in the same
 run, one block each in the same JSON line: paged decode ("decode": batch 32,

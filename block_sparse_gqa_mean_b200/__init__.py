@@ -348,10 +348,10 @@ def sparse_attn_decode_noalloc(cache: PagedKVCache, q: torch.Tensor, block_idx: 
                                out: torch.Tensor, lse: Optional[torch.Tensor] = None,
                                softmax_scale: Optional[float] = None, stream=None):
     """sparse_attn_decode for callers that cannot allocate device memory: the
-    caller passes the outputs, and the split-k scratch is the library's own
-    8 MiB device array (shared by every call on the device, so calls must not
-    overlap on the GPU). Raises MsaError(MSA_ERR_WORKSPACE) when the problem
-    needs more scratch than that."""
+    caller passes the outputs, and the attention's scratch (one part and flag
+    per resident CTA, at most ~5 MiB) is the library's own 8 MiB device array
+    (shared by every call on the device, so calls must not overlap on the
+    GPU)."""
     lib = load_library()
     _require_cuda(q, block_idx, out, lse)
     top_k = block_idx.shape[-1]

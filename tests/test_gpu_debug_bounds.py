@@ -5,7 +5,7 @@ loads libmsa_debug.so (MSA_LIBRARY) and runs there:
   * parity cases against the oracle that reach every kernel family (append
     and pooling, prefill selection, decode pass 1 and merge, the tcgen05
     prefill attention with its clustering and plan kernels, the SIMT path,
-    split-k decode, the token variant, the context-sharded decode), each of
+    decode attention, the token variant, the context-sharded decode), each of
     which also asserts a clean status word: no check fires on valid input;
   * the two tests below, which break a launch-size precondition that the
     regular build cannot see (the caller's max rows / max new tokens per

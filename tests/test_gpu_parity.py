@@ -307,7 +307,7 @@ DECODE_CASES = [
 
 
 def test_decode_repeated_and_empty_block_lists():
-    """Split-k decode: an adjacent repeat of a block counts once, a sequence
+    """Decode attention: an adjacent repeat of a block counts once, a sequence
     whose list is all -1 gives 0 and lse = -inf."""
     w = workloads.paged_decode_bf16(batch=3, ctx=(3000, 5000, 4096))
     p = workloads.paging(w)
