@@ -4,9 +4,10 @@ The oracle checks sampled outputs it can compute one by one:
   * prefill (batch 1, 32768 tokens, 32/4 heads, d 128, block 128, top-k 16):
     288 rows spread across the sequence, most of them at block edges (the
     first, second and last token of a block) and the rest at random;
-  * paged decode (batch 32 x 131072 cached tokens, block 64, top-k 32) and
-    varlen decode (64 sequences of 4K-512K tokens, block 64, top-k 64): whole
-    sampled sequences;
+  * paged decode (batch 32 x 131072 cached tokens, block 64, top-k 32; 8 of
+    the 32 sequences) and varlen decode (64 sequences of 4K-512K tokens,
+    block 64, top-k 64; the shortest, the longest and four lengths between):
+    whole sampled sequences;
   * 1M-context decode (1048576 cached tokens, block 128, top-k 16): all 256
     consecutive decode steps run, each appending one token; at steps 0, 127,
     128 (the first token of a new block) and 255 the oracle rebuilds every
@@ -76,14 +77,15 @@ def _decode_step(w, cache):
 
 
 @pytest.mark.parametrize("make,seqs", [
-    (workloads.paged_decode_bf16, (0, 31)),
+    (workloads.paged_decode_bf16, (0, 5, 11, 15, 19, 23, 27, 31)),
     (workloads.varlen_decode_bf16, None),
 ], ids=["paged_decode", "varlen_decode"])
 def test_full_decode_sampled_sequences(make, seqs):
     w = make()
-    if seqs is None:  # the shortest and a middle-length sequence
+    if seqs is None:  # the shortest, the longest and four lengths between, by rank
         order = np.argsort(np.array(w.ctx))
-        seqs = (int(order[0]), int(order[len(order) // 2]))
+        n = len(order)
+        seqs = tuple(int(order[i]) for i in (0, n // 5, 2 * n // 5, 3 * n // 5, 4 * n // 5, n - 1))
     p = workloads.paging(w)
     cache = new_cache(w, p)
     lens, q, idx, out = _decode_step(w, cache)
