@@ -55,7 +55,7 @@ __global__ void __launch_bounds__(128) append_pool_kernel(
   const int u_lo = max(t0, j * B);
   const int u_hi = min(L, (j + 1) * B);
   const size_t page_off = ((size_t)page * hkv + g) * B * D;
-  const size_t pool = (size_t)num_pages * hkv * B * D;
+  [[maybe_unused]] const size_t pool = (size_t)num_pages * hkv * B * D;  // bounds-checked build
   extern __shared__ __align__(16) unsigned char smem_raw[];
   T* tile = reinterpret_cast<T*>(smem_raw);  // [n][D]
 
