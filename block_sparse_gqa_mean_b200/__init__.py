@@ -43,7 +43,7 @@ EXPORTS = ("msa_build_block_cache", "msa_select_topk", "msa_sparse_attn_prefill"
            "msa_status_string", "msa_version", "msa_select_tokens", "msa_sparse_attn_decode_tokens",
            "msa_select_topk_range", "msa_select_merge", "msa_sparse_attn_decode_range",
            "msa_lse_merge", "msa_select_tokens_rows", "msa_sparse_attn_prefill_tokens",
-           "msa_build_flags")
+           "msa_build_flags", "msa_selftest_bounded_wait")
 
 
 class MsaError(RuntimeError):
@@ -110,6 +110,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.msa_status_string.restype = ctypes.c_char_p
     lib.msa_version.restype = I32
     lib.msa_build_flags.restype = I32
+    lib.msa_selftest_bounded_wait.argtypes = [I32, P, P]
+    lib.msa_selftest_bounded_wait.restype = ctypes.c_int
     for name in ("msa_build_block_cache", "msa_select_topk", "msa_sparse_attn_prefill",
                  "msa_sparse_attn_decode", "msa_sparse_attn_prefill_gated",
                  "msa_sparse_attn_decode_gated", "msa_sparse_attn_decode_noalloc",
@@ -123,6 +125,16 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
 
 def status_string(status: int) -> str:
     return load_library().msa_status_string(status).decode()
+
+
+def selftest_bounded_wait(which: int, status_word: torch.Tensor, stream=None) -> None:
+    """Run one of the library's bounded device waits on something that is
+    never completed (0: an mbarrier phase, 1: a flag another CTA would
+    publish); after about a second it sets MSA_DEV_TIMEOUT in status_word
+    (a one-element int32 CUDA tensor) and returns."""
+    _require_cuda(status_word)
+    _check(load_library().msa_selftest_bounded_wait(int(which), _ptr(status_word), _stream(stream)),
+           "msa_selftest_bounded_wait")
 
 
 def build_flags() -> int:

@@ -60,15 +60,6 @@ constexpr float kLn2 = 0.6931471805599453f;
 constexpr int kStreamNST = 2;  // pipeline stages
 using namespace warpmma;
 
-__device__ __forceinline__ uint64_t ld_acquire_u64(const uint64_t* p) {
-  uint64_t v;
-  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-  return v;
-}
-__device__ __forceinline__ void st_release_u64(uint64_t* p, uint64_t v) {
-  asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
-}
-
 // The CTA whose range holds slot x (the largest c with c W / C <= x).
 __device__ __forceinline__ int cta_of_slot(long long x, int C, long long W) {
   return (int)(((x + 1) * C - 1) / W);
@@ -341,14 +332,9 @@ __global__ void __launch_bounds__(128, B == 64 ? 3 : 1) decode_streamk_kernel(
     if (np > 0) {
       const uint64_t t0 = global_timer_ns();
       for (int k = tid; k < np && ok; k += 128) {
-        uint32_t spins = 0;
-        while (ld_acquire_u64(flags + c + 1 + k) != tag) {
-          if ((++spins & 63u) == 0 && global_timer_ns() - t0 > 1000000000ull) {
-            report(status, MSA_DEV_TIMEOUT);
-            ok = 0;
-            break;
-          }
-          __nanosleep(32);
+        if (!wait_flag(flags + c + 1 + k, tag, t0)) {
+          report(status, MSA_DEV_TIMEOUT);
+          ok = 0;
         }
       }
     }

@@ -35,6 +35,7 @@ cudaError_t select_merge_lists(const msa_paged_kv_t*, const uint64_t*, int, int,
 cudaError_t decode_splitk_range(const msa_paged_kv_t*, const void*, const int32_t*, int, float,
                                 float*, float*, void*, int, int, int, cudaStream_t);
 cudaError_t lse_merge(const float*, const float*, int, int, int, bool, void*, float*, cudaStream_t);
+cudaError_t selftest_wait(int which, uint32_t* status, cudaStream_t st);
 bool prefill_tc_supported(const msa_paged_kv_t*);
 size_t prefill_ws(const msa_paged_kv_t*, int max_rows, int top_k);
 cudaError_t prefill_tc(const msa_paged_kv_t*, const void*, const int32_t*, int, const int32_t*,
@@ -134,6 +135,13 @@ extern "C" {
 int32_t msa_version(void) { return 1000; }
 
 int32_t msa_build_flags(void) { return kDebugBounds ? MSA_BUILD_DEBUG_BOUNDS : 0; }
+
+msa_status_t msa_selftest_bounded_wait(int32_t which, uint32_t* status_word,
+                                       msa_stream_t stream) {
+  if (!status_word || !aligned(status_word, 4) || (which != 0 && which != 1))
+    return MSA_ERR_INVALID_ARG;
+  return from_cuda(selftest_wait(which, status_word, (cudaStream_t)stream));
+}
 
 const char* msa_status_string(msa_status_t s) {
   switch (s) {

@@ -62,6 +62,26 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   return false;
 }
 
+// Flags that one CTA publishes for another (release store / acquire load at
+// GPU scope), and a bounded wait for a flag to carry `tag`: false once about
+// one second of %globaltimer time since t0 has passed.
+__device__ __forceinline__ uint64_t ld_acquire_u64(const uint64_t* p) {
+  uint64_t v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_u64(uint64_t* p, uint64_t v) {
+  asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+__device__ __forceinline__ bool wait_flag(const uint64_t* flag, uint64_t tag, uint64_t t0) {
+  uint32_t spins = 0;
+  while (ld_acquire_u64(flag) != tag) {
+    if ((++spins & 63u) == 0 && global_timer_ns() - t0 > 1000000000ull) return false;
+    __nanosleep(32);
+  }
+  return true;
+}
+
 // 2-D tiled TMA load (no multicast) completing on `bar` with complete_tx.
 // x is the innermost coordinate in elements; callers keep x * elem_size a
 // multiple of 16 bytes.

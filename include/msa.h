@@ -450,6 +450,19 @@ int32_t msa_version(void);
 #define MSA_BUILD_DEBUG_BOUNDS 0x1
 int32_t msa_build_flags(void);
 
+/* Self-test of the bounded device waits. Every wait of the library's kernels
+ * on another agent (an mbarrier phase completed by TMA copies or other warps,
+ * a flag another CTA publishes) gives up after about one second, sets
+ * MSA_DEV_TIMEOUT in the status word and lets the kernel return. This call
+ * launches one small kernel that runs such a wait on something never
+ * completed - which = 0: an mbarrier phase nothing arrives at; which = 1: a
+ * flag word nothing writes - so that after about one second *status_word has
+ * MSA_DEV_TIMEOUT set and the context is still usable.
+ *   status_word : device pointer to a uint32 (4-byte aligned).
+ * Returns MSA_ERR_INVALID_ARG for a NULL or misaligned status_word or which
+ * not 0 or 1, MSA_ERR_CUDA if the launch fails. */
+msa_status_t msa_selftest_bounded_wait(int32_t which, uint32_t* status_word, msa_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -43,6 +43,13 @@ def test_struct_layout_matches_header():
     assert msa._PagedKV.status_word.offset == 32 + 5 * 8
 
 
+def test_selftest_rejects_bad_arguments_without_a_gpu():
+    lib = msa.load_library()
+    assert lib.msa_selftest_bounded_wait(0, None, None) == msa.MSA_ERR_INVALID_ARG
+    assert lib.msa_selftest_bounded_wait(2, 4096, None) == msa.MSA_ERR_INVALID_ARG
+    assert lib.msa_selftest_bounded_wait(1, 4098, None) == msa.MSA_ERR_INVALID_ARG  # misaligned
+
+
 def test_null_cache_is_rejected_without_a_gpu():
     lib = msa.load_library()
     assert lib.msa_select_topk(None, None, None, 1, 1, 4, None, None, None, 0, None) == \

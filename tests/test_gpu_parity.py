@@ -497,3 +497,36 @@ def test_decode_graph_replays_and_shared_workspace(name, make):
     torch.cuda.synchronize()
     assert torch.equal(_bits(out0), _bits(ref0))
     assert cache.device_status() == 0
+
+
+@pytest.mark.parametrize("which", [0, 1], ids=["mbarrier_phase", "published_flag"])
+def test_bounded_wait_gives_up_and_context_survives(which):
+    """A device wait on something never completed (an mbarrier phase nothing
+    arrives at, a flag nothing publishes) gives up after about a second with
+    MSA_DEV_TIMEOUT, and the context keeps working: a decode step afterwards
+    matches the oracle."""
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    msa.selftest_bounded_wait(which, st)
+    b.record()
+    torch.cuda.synchronize()
+    assert st.item() == msa.MSA_DEV_TIMEOUT
+    assert 900.0 <= a.elapsed_time(b) <= 5000.0
+    w = workloads.paged_decode_bf16(batch=2, ctx=(500, 700))
+    p = workloads.paging(w)
+    cache = new_cache(w, p)
+    lens = fill_context(cache, w)
+    after = [L + 1 for L in lens]
+    append(cache, w, lens, after)
+    q = workloads.queries_decode(w, 0, DEV)
+    idx, _ = msa.select_topk(cache, q, w.top_k)
+    out, _ = msa.sparse_attn_decode(cache, q, idx)
+    torch.cuda.synchronize()
+    assert cache.device_status() == 0
+    for bq in range(w.batch):
+        L = after[bq]
+        K, V = workloads.keys(w, bq, 0, L), workloads.values(w, bq, 0, L)
+        O, _ = oracle.attend(q[bq:bq + 1].cpu(), K, V, np.array([L - 1]),
+                             idx[bq:bq + 1].cpu().numpy(), w.block, w.softmax_scale)
+        compare(out[bq:bq + 1], O, "bf16")
